@@ -215,7 +215,9 @@ def rmsnorm(x, norm_w, eps: float):
     """
     x = np.asarray(x, dtype=np.float64)
     e = float(np.float32(eps))
-    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1) + e)
+    ms = np.mean(x * x, axis=-1) + e
+    # an all-zero row with eps = 0 stays zero (scale 0, codes 0) instead of 0/0
+    r = np.where(ms > 0, 1.0 / np.sqrt(np.where(ms > 0, ms, 1.0)), 0.0)
     return x * r[..., None] * (1.0 + np.asarray(norm_w, dtype=np.float64))[None, :]
 
 

@@ -358,3 +358,11 @@ def test_int4_row_error_plausible_against_card():
     deq = out["codes"].astype(np.float64) * out["s64"][:, None]
     rel = np.linalg.norm(out["rotated"] - deq, axis=1) / np.linalg.norm(out["rotated"], axis=1)
     assert abs(rel.mean() - card) < 0.03
+
+
+def test_zero_row_with_zero_eps_stays_zero():
+    x = np.zeros((2, 256))
+    x[1, 3] = 1.0
+    q, s, v = ref.rotate_quant_act(x, norm_w=np.zeros(256), eps=0.0)
+    assert s[0] == 0.0 and not q[0].any() and np.isfinite(v).all()
+    assert s[1] > 0
