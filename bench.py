@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the ConvRot W8A8 linear on B200.
+
+One step = one pass of the per-token hot path over one batch of synthetic
+input: the rotate-quantise kernel (with the fused RMSNorm when the workload has
+one) and the tcgen05 W8A8 GEMM with its dequant epilogue.  Weight preparation
+(SmoothQuant calibration, rotation, per-row quantisation) is offline and not
+timed.  The default workload is the down-proj shaped linear: 512 tokens,
+K = 12288, N = 4096, RMSNorm with folded SmoothQuant scales.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, timed on the host
+
+Under torchrun every rank runs an independent replica (the linear has no data
+exchange); the timed region is bracketed by barriers and the max over ranks
+is reported.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "ConvRot W8A8 linear TOPS and tokens/s vs INT8 tensor & HBM roofline"
+DEFAULT_WORKLOAD = "down_proj_m512"
+# dense int8 tensor peak = measured dense bf16 peak x the nominal int8:bf16 ratio (4.5 / 2.25)
+INT8_PER_BF16 = 2.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "w8a8_int8_quantized_rmsnorm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(workload, {}).get(kernel)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+class Linear:
+    def __init__(self, lin, Wq, s_row, group_in):
+        self.lin = lin
+        self.Wq = Wq
+        self.s_row = s_row
+        self.group_in = group_in
+
+
+def input_groups(w):
+    """Linears that read the same activation share one rotate-quantise call."""
+    groups = []
+    for lin in w.linears:
+        key = {"q_proj": "attn", "k_proj": "attn", "v_proj": "attn", "o_proj": "o",
+               "gate_proj": "mlp", "up_proj": "mlp", "down_proj": "down"}.get(lin.name, lin.name)
+        for g in groups:
+            if g["key"] == key:
+                g["linears"].append(lin)
+                break
+        else:
+            groups.append({"key": key, "K": lin.K, "linears": [lin]})
+    return groups
+
+
+def prepare(cr, w, dev):
+    """Synthetic inputs and offline weight preparation (untimed)."""
+    groups = input_groups(w)
+    inputs, norms = [], []
+    for gi, g in enumerate(groups):
+        lin0 = g["linears"][0]
+        x = workloads.activations(w.M, lin0.K, dist=w.dist, outlier_count=w.n_outliers(lin0.K),
+                                  outlier_scale=w.outlier_scale)
+        nw = workloads.norm_weight(lin0.K) if w.norm else None
+        inputs.append(x.to(dev))
+        norms.append(None if nw is None else nw.to(dev))
+    raw_norms = list(norms)
+    layers = []
+    for layer in range(w.layers):
+        for gi, g in enumerate(groups):
+            for lin in g["linears"]:
+                gen_dev = "cpu" if lin.N * lin.K <= (1 << 27) and w.layers == 1 else dev
+                W = workloads.weight(lin.N, lin.K, layer=layer, device=gen_dev).to(dev)
+                col = None
+                if raw_norms[gi] is not None:
+                    # one norm-carrying linear per input group in these workloads
+                    col, norms[gi] = cr.convrot_smoothquant_calibrate(inputs[gi], raw_norms[gi], W)
+                if w.weight_bits == 8:
+                    Wq, s_row = cr.convrot_quantize_weight(W, 256, col)
+                else:
+                    Wq, s_row = cr.convrot_quantize_weight_w4(W, 256, col)
+                del W
+                layers.append(Linear(lin, Wq, s_row, gi))
+    torch.cuda.synchronize(dev)
+    return groups, inputs, norms, layers
+
+
+def run_ours(args, rank, world, dev):
+    import w8a8_int8_quantized_rmsnorm_b200 as cr
+    cr.lib()
+    w = workloads.WORKLOADS[args.workload]
+    peaks = load_peaks()
+    torch.cuda.set_device(dev)
+    groups, inputs, norms, layers = prepare(cr, w, dev)
+
+    # copies of the per-step operands so that no step finds its inputs in L2
+    step_bytes = sum(x.numel() * 2 for x in inputs) + sum(l.Wq.numel() for l in layers)
+    copies = 1 if step_bytes > 2 * L2_BYTES else min(8, math.ceil(3 * L2_BYTES / step_bytes))
+    x_sets = [inputs] + [[x.clone() for x in inputs] for _ in range(copies - 1)]
+    w_sets = [[(l.Wq, l.s_row) for l in layers]] + \
+             [[(l.Wq.clone(), l.s_row.clone()) for l in layers] for _ in range(copies - 1)]
+    ws = cr.Workspace(dev.index)
+    Xq = [torch.empty(w.M, g["K"], dtype=torch.int8, device=dev) for g in groups]
+    st = [torch.empty(w.M, dtype=torch.float32, device=dev) for g in groups]
+    Ys = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16, device=dev) for l in layers]
+    linear = cr.convrot_int8_linear if w.weight_bits == 8 else cr.convrot_w4a8_linear
+
+    stream = torch.cuda.current_stream(dev)
+    n_k1 = len(groups)
+    n_k2 = len(layers)
+
+    def step(i, ev=None):
+        c = i % copies
+        for gi in range(n_k1):
+            if ev is not None:
+                ev[0][gi].record(stream)
+            cr.convrot_rotate_quant_act(x_sets[c][gi], 256, norms[gi], 1e-6, out=(Xq[gi], st[gi]))
+            if ev is not None:
+                ev[1][gi].record(stream)
+        for li, l in enumerate(layers):
+            if ev is not None:
+                ev[2][li].record(stream)
+            Wq, s_row = w_sets[c][li]
+            linear(Xq[l.group_in], st[l.group_in], Wq, s_row, out=Ys[li], workspace=ws)
+            if ev is not None:
+                ev[3][li].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    status = cr.convrot_device_status(dev.index)
+    if status:
+        raise RuntimeError(f"device error word {status:#x} after warm-up")
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    per_step_events = [[events(n_k1), events(n_k1), events(n_k2), events(n_k2)]
+                       for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, per_step_events[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = cr.convrot_device_status(dev.index)
+    if status:
+        raise RuntimeError(f"device error word {status:#x} in the timed region")
+
+    k1_ms = [sum(e[0][g].elapsed_time(e[1][g]) for g in range(n_k1)) for e in per_step_events]
+    k2_ms = [sum(e[2][l].elapsed_time(e[3][l]) for l in range(n_k2)) for e in per_step_events]
+    k1_avg = statistics.mean(k1_ms) / n_k1  # per launch
+    k2_avg = statistics.mean(k2_ms) / n_k2
+
+    tokens = w.M * args.steps * world
+    ops = w.ops() * args.steps * world
+    secs = elapsed_ms / 1e3
+    k1_bytes = sum(w.M * g["K"] * 3 + 4 * w.M + (4 * g["K"] if w.norm else 0) for g in groups)
+    k2_bytes = sum(w.M * l.lin.K + l.Wq.numel() + 2 * w.M * l.lin.N + 4 * (w.M + l.lin.N)
+                   for l in layers)
+    k2_ops = w.ops()
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    k2_achieved_tops = k2_ops / (statistics.mean(k2_ms) / 1e3) / 1e12
+    k2_achieved_gbs = k2_bytes / (statistics.mean(k2_ms) / 1e3) / 1e9
+    k1_achieved_gbs = k1_bytes / (statistics.mean(k1_ms) / 1e3) / 1e9
+    # the GEMM dominates every workload's step; it is tensor-bound above the
+    # ridge (~250 tokens) and weight-stream (HBM) bound below it
+    ridge_bound = "tensor" if w.M > 256 else "hbm"
+    if ridge_bound == "tensor":
+        roof = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::i8)",
+                "achieved": round(k2_achieved_tops, 1), "peak": round(int8_peak, 1),
+                "unit": "TOP/s", "frac": round(k2_achieved_tops / int8_peak, 4),
+                "peak_note": f"{peaks['source']}: 2 x dense bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "kernel": "gemm_kernel (tcgen05 kind::i8)",
+                "achieved": round(k2_achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(k2_achieved_gbs / peaks["hbm_gbs"], 4),
+                "peak_note": f"{peaks['source']} copy bandwidth"}
+    roof["traffic"] = profiled_traffic("gemm_kernel", args.workload)
+    roof["algorithmic_per_launch"] = (k2_ops / n_k2) if ridge_bound == "tensor" else (k2_bytes / n_k2)
+
+    result = {
+        "metric": METRIC,
+        "value": round(tokens / secs, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "i8",
+        "data": "synthetic (seeded; no trained weights or datasets)",
+        "tops": round(ops / secs / 1e12, 1),
+        "config": {
+            "workload": args.workload, "M": w.M,
+            "linears": [[l.name, l.N, l.K] for l in w.linears], "layers": w.layers,
+            "weight_bits": w.weight_bits, "group": 256, "rmsnorm": w.norm,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": (f"{copies} rotating copies of the step's inputs "
+                   f"({copies * step_bytes / 1e6:.0f} MB > L2)") if copies > 1
+                  else f"step inputs {step_bytes / 1e6:.0f} MB > 2x L2",
+        },
+        "roofline": roof,
+        "kernels": {
+            "rotate_quant_act": {"launches_per_step": n_k1, "avg_us": round(k1_avg * 1e3, 3),
+                                 "bound": "hbm", "achieved_GBps": round(k1_achieved_gbs, 1),
+                                 "frac": round(k1_achieved_gbs / peaks["hbm_gbs"], 4),
+                                 "algorithmic_bytes_per_step": k1_bytes},
+            "gemm": {"launches_per_step": n_k2, "avg_us": round(k2_avg * 1e3, 3),
+                     "achieved_TOPs": round(k2_achieved_tops, 1),
+                     "tensor_frac": round(k2_achieved_tops / int8_peak, 4),
+                     "achieved_GBps": round(k2_achieved_gbs, 1),
+                     "hbm_frac": round(k2_achieved_gbs / peaks["hbm_gbs"], 4),
+                     "algorithmic_bytes_per_step": k2_bytes, "ops_per_step": k2_ops},
+        },
+        "gpu_launches": (n_k1 + n_k2) * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_e2e:
+        result["e2e"] = e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world)
+    return result
+
+
+def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
+    """Same metric through the public API with pinned host buffers: each step
+    copies its activations host->device and its outputs device->host."""
+    host_x = [x.cpu().pin_memory() for x in inputs]
+    host_y = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16).pin_memory() for l in layers]
+    ws = cr.Workspace(dev.index)
+    linear = cr.convrot_int8_linear if w.weight_bits == 8 else cr.convrot_w4a8_linear
+    stream = torch.cuda.current_stream(dev)
+    steps = max(5, min(args.steps, 50))
+
+    def step():
+        xs = [h.to(dev, non_blocking=True) for h in host_x]
+        qs = [cr.convrot_rotate_quant_act(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
+        for li, l in enumerate(layers):
+            Y = linear(qs[l.group_in][0], qs[l.group_in][1], l.Wq, l.s_row, workspace=ws)
+            host_y[li].copy_(Y, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(w.M * steps * world / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": sum(h.numel() * 2 for h in host_x),
+            "d2h_bytes_per_step": sum(h.numel() * 2 for h in host_y), "steps": steps}
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_step_runner(w, sample_tokens):
+    """Prepares the oracle's weights (untimed) and returns a callable that runs
+    the oracle's per-token path on `sample_tokens` tokens of the workload."""
+    from oracle import convrot_ref as ref
+    groups = input_groups(w)
+    xs, nws, preps = [], [], []
+    for g in groups:
+        lin0 = g["linears"][0]
+        x, _, nw = workloads.workload_inputs(w, lin0, M=min(w.M, max(sample_tokens, 1)))
+        xs.append(x.float().double().numpy()[:sample_tokens])
+        nws.append(None if nw is None else nw.double().numpy())
+    for gi, g in enumerate(groups):
+        for lin in g["linears"]:
+            W = workloads.weight(lin.N, lin.K).float().double().numpy()
+            col = None
+            if nws[gi] is not None:
+                col, nws[gi] = ref.smoothquant_scales(xs[gi], nws[gi], 1e-6, W)
+            if w.weight_bits == 8:
+                Wq, s_row, _ = ref.quantize_weight(W, 256, col)
+                preps.append((gi, Wq, s_row, None))
+            else:
+                o = ref.quantize_weight_w4(W, 256, col)
+                preps.append((gi, None, o["s_row"], o["packed"]))
+
+    def run():
+        acts = [ref.rotate_quant_act(xs[g], 256, nws[g], 1e-6) for g in range(len(groups))]
+        for gi, Wq, s_row, packed in preps:
+            Xq, s_tok, _ = acts[gi]
+            if packed is None:
+                ref.int8_linear(Xq, s_tok, Wq, s_row)
+            else:
+                ref.w4a8_linear(Xq, s_tok, packed, s_row)
+    return run
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, target_s=10.0):
+    """The oracle as it stands on the host cores, on a bounded sample."""
+    sample = min(w.M, 64 if w.layers == 1 else 16)
+    run = oracle_step_runner(w, sample)
+    run()  # warm
+    reps, t = 0, 0.0
+    t0 = time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        t = time.perf_counter() - t0
+        if t >= target_s or reps >= 1000:
+            break
+    per_tok = t / (reps * sample * w.layers)
+    return {"value": round(1.0 / per_tok, 2), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{sample} tokens of {w.name} x {reps} repetitions "
+                      f"({t:.1f} s; float64 numpy, every linear of the step"
+                      + (f", 1 of {w.layers} layers, scaled" if w.layers > 1 else "") + ")"}
+
+
+def run_reference(args, rank, world):
+    w = workloads.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    sample = min(w.M, 64 if w.layers == 1 else 16)
+    run = oracle_step_runner(w, sample)
+    for _ in range(max(1, min(args.warmup, 3))):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    secs = time.perf_counter() - t0
+    tok_s = sample * args.steps / secs / w.layers
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(tok_s, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "M": w.M, "sample_tokens_per_step": sample},
+        "cpu_baseline": {"value": round(tok_s, 2), "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{sample} tokens of {w.name} per step"},
+        "e2e": {"value": round(tok_s, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[args.workload])
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

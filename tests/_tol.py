@@ -1,0 +1,81 @@
+"""Tolerances of the CUDA path against the float64 oracle, derived from the
+fp32 arithmetic the kernels perform.
+
+The kernels take every rounding decision in fp32 while the oracle takes it in
+float64.  A code can therefore differ only where the oracle's value lies
+within the fp32 error of a rounding tie; these helpers bound that error.
+
+Error model (u = 2^-24, unit roundoff of fp32):
+* inputs: bf16 values are exact in fp32; a per-column multiplier (RMSNorm
+  weight 1 + w, or a column scale) adds at most 2u relative per element;
+* FWHT: 8 butterfly stages, each stage's rounding error is at most u times the
+  2-norm of that stage's output, and later stages scale errors by sqrt(2) per
+  stage like the signal, so the error of a group's transform has 2-norm at
+  most 8u * ||v_g||_2 (plus 2u * ||v_g||_2 from the inputs);
+* per-row absmax: off by at most E = max_g 10u ||v_g||_2;
+* codes: z = v * fp32(127 / absmax), two more roundings.
+A factor of 1.5 covers second-order terms.
+"""
+import numpy as np
+
+U = 2.0 ** -24
+
+
+def row_error(v, group, pre):
+    """E / absmax per row (0 for all-zero rows), for the rotated values v."""
+    v = np.asarray(v, dtype=np.float64)
+    amax = np.max(np.abs(v), axis=1)
+    if group:
+        M, K = v.shape
+        gn = np.sqrt(np.sum(v.reshape(M, K // group, group) ** 2, axis=2)).max(axis=1)
+        E = (8.0 + (2.0 if pre else 0.0)) * U * gn
+    else:
+        E = (2.0 * U if pre else 0.0) * amax
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.where(amax > 0, E / np.where(amax > 0, amax, 1.0), 0.0)
+    return r, amax
+
+
+def int8_code_window(ratio):
+    """Half-width of the window around a tie in which an int8 code may flip."""
+    return 1.5 * 127.0 * (2.0 * ratio + 2.0 * U)
+
+
+def scale_rel_tol(ratio, norm):
+    """Relative tolerance of the fp32 per-row scale against float64."""
+    return 1.5 * (ratio + (5.0 if norm else 1.0) * U) + 2.0 * U
+
+
+def check_codes(q_gpu, q_ref, z, window, name="codes"):
+    """|q_gpu - q_ref| <= 1, and only where |frac(|z|) - 1/2| <= window (per row).
+
+    Returns the number of differing codes.
+    """
+    q_gpu = np.asarray(q_gpu, dtype=np.int64)
+    q_ref = np.asarray(q_ref, dtype=np.int64)
+    diff = q_gpu - q_ref
+    assert np.abs(diff).max(initial=0) <= 1, f"{name}: a code differs by more than 1"
+    az = np.abs(z)
+    dist = np.abs(az - np.floor(az) - 0.5)
+    w = np.broadcast_to(np.asarray(window, dtype=np.float64)[:, None], dist.shape)
+    bad = (diff != 0) & (dist > w)
+    if bad.any():
+        i, j = np.argwhere(bad)[0]
+        raise AssertionError(f"{name}: code differs away from a tie at ({i},{j}): "
+                             f"z={z[i, j]!r} gpu={q_gpu[i, j]} ref={q_ref[i, j]} "
+                             f"dist={dist[i, j]:.3e} window={w[i, j]:.3e}")
+    return int((diff != 0).sum())
+
+
+def bf16_ulp(y):
+    """Spacing of bfloat16 numbers at |y| (2^(e-7) for 2^e <= |y| < 2^(e+1))."""
+    y = np.abs(np.asarray(y, dtype=np.float64))
+    _, e = np.frexp(np.where(y > 0, y, 1.0))
+    e = np.maximum(e - 1, -126)
+    return np.ldexp(1.0, e - 7)
+
+
+def output_tol(y_ref):
+    """Output tolerance: |y - y_ref| <= 2^-7 |y_ref| + 1e-3 max_n |y_ref[m, :]|."""
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    return 2.0 ** -7 * np.abs(y_ref) + 1e-3 * np.max(np.abs(y_ref), axis=1, keepdims=True)

@@ -1,0 +1,145 @@
+"""Parity of the tcgen05 W8A8 / W4A8 GEMM kernels with the oracle, through the
+C ABI: int32 accumulators bit-exact, bf16 outputs within one bf16 rounding of
+the float64 dequantisation, over shapes that exercise both operand roles,
+ragged tails in M, N and K, data-parallel and stream-K schedules."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import convrot_ref as ref
+from tests import _tol
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cr():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import w8a8_int8_quantized_rmsnorm_b200 as m
+    m.lib()
+    return m
+
+
+def _rand_i8(shape, seed, lo=-128, hi=128):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(lo, hi, shape, generator=g, dtype=torch.int16).to(torch.int8)
+
+
+def _rand_scales(n, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand(n, generator=g, dtype=torch.float64) * 1e-3 + 1e-5).float()
+
+
+SHAPES = [
+    # (M, N, K): operand roles swap at M <= 128
+    (1, 256, 512), (3, 136, 512), (16, 1024, 4096), (17, 264, 1040), (40, 512, 256),
+    (64, 128, 768), (100, 2056, 144), (128, 520, 4096),
+    (129, 264, 512), (256, 512, 4096), (300, 1032, 1040), (512, 4096, 12288),
+    (1024, 1024, 4096), (2048, 1536, 16), (777, 8, 32),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_int8_gemm_s32_bit_exact(cr, M, N, K):
+    X = _rand_i8((M, K), M * 31 + K)
+    W = _rand_i8((N, K), N * 17 + K)
+    acc = cr.convrot_int8_gemm_s32(X.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    assert cr.convrot_device_status() == 0
+    want = ref.int_matmul(X.numpy(), W.numpy())
+    got = acc.cpu().numpy().astype(np.int64)
+    assert np.array_equal(got, want), f"{np.count_nonzero(got != want)} mismatches"
+
+
+def test_int8_gemm_s32_extreme_operands(cr):
+    M, N, K = 130, 264, 12288
+    X = torch.full((M, K), 127, dtype=torch.int8)
+    X[1::2] = -127
+    W = torch.full((N, K), -127, dtype=torch.int8)
+    W[::3, ::2] = 127
+    acc = cr.convrot_int8_gemm_s32(X.cuda(), W.cuda()).cpu().numpy()
+    assert np.array_equal(acc.astype(np.int64), ref.int_matmul(X.numpy(), W.numpy()))
+    assert acc[0, 1] == -127 * 127 * K
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES[:-1])
+def test_int8_linear_bf16(cr, M, N, K):
+    X = _rand_i8((M, K), M + 5 * K, -127, 128)
+    W = _rand_i8((N, K), N + 3 * K, -127, 128)
+    st = _rand_scales(M, 1)
+    sr = _rand_scales(N, 2)
+    Y = cr.convrot_int8_linear(X.cuda(), st.cuda(), W.cuda(), sr.cuda())
+    torch.cuda.synchronize()
+    yb, y64, _ = ref.int8_linear(X.numpy(), st.double().numpy(), W.numpy(), sr.double().numpy())
+    got = Y.float().cpu().double().numpy()
+    # fp32 product then one bf16 rounding: at most one bf16 step from the
+    # correctly rounded float64 value
+    assert np.all(np.abs(got - yb) <= _tol.bf16_ulp(y64) * 1.0001)
+
+
+PACK_SHAPES = [(1, 256, 512), (16, 1024, 4096), (33, 264, 1056), (128, 520, 4096),
+               (129, 264, 512), (512, 4096, 12288), (1000, 1032, 2080)]
+
+
+def _rand_w4(N, K, seed):
+    codes = torch.randint(-8, 8, (N, K), generator=torch.Generator().manual_seed(seed))
+    packed = ref.pack_int4(codes.numpy())
+    return codes.numpy().astype(np.int8), torch.from_numpy(packed)
+
+
+@pytest.mark.parametrize("M,N,K", PACK_SHAPES)
+def test_w4a8_gemm_s32_bit_exact(cr, M, N, K):
+    X = _rand_i8((M, K), 7 * M + K)
+    codes, packed = _rand_w4(N, K, N + K)
+    acc = cr.convrot_w4a8_gemm_s32(X.cuda(), packed.cuda())
+    torch.cuda.synchronize()
+    assert cr.convrot_device_status() == 0
+    want = ref.int_matmul(X.numpy(), ref.unpack_int4(packed.numpy()))
+    assert np.array_equal(codes, ref.unpack_int4(packed.numpy()))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), want)
+
+
+@pytest.mark.parametrize("M,N,K", PACK_SHAPES)
+def test_w4a8_linear_bf16(cr, M, N, K):
+    X = _rand_i8((M, K), M + K, -127, 128)
+    _, packed = _rand_w4(N, K, 3 * N + K)
+    st = _rand_scales(M, 3)
+    sr = _rand_scales(N, 4)
+    Y = cr.convrot_w4a8_linear(X.cuda(), st.cuda(), packed.cuda(), sr.cuda())
+    torch.cuda.synchronize()
+    yb, y64, _ = ref.w4a8_linear(X.numpy(), st.double().numpy(), packed.numpy(), sr.double().numpy())
+    got = Y.float().cpu().double().numpy()
+    assert np.all(np.abs(got - yb) <= _tol.bf16_ulp(y64) * 1.0001)
+
+
+def test_workspace_reuse_and_determinism(cr):
+    # this shape splits tiles by K across CTAs, so partial tiles meet in the
+    # workspace; reusing it for further calls only gives the right answer if
+    # every call restores the tile counters to zero
+    M, N, K = 512, 4096, 12288
+    assert cr.convrot_linear_workspace_bytes(M, N, K, 8) > 0
+    ws = cr.Workspace()
+    X = _rand_i8((M, K), 11)
+    W = _rand_i8((N, K), 12)
+    want = ref.int_matmul(X.numpy(), W.numpy())
+    Xd, Wd = X.cuda(), W.cuda()
+    for _ in range(3):
+        acc = cr.convrot_int8_gemm_s32(Xd, Wd, workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64), want)
+    assert int(ws.buf[-256:].count_nonzero().item()) == 0
+
+
+def test_workspace_too_small_is_rejected(cr):
+    M, N, K = 512, 4096, 12288
+    X = torch.zeros(M, K, dtype=torch.int8, device="cuda")
+    W = torch.zeros(N, K, dtype=torch.int8, device="cuda")
+    s = torch.ones(max(M, N), device="cuda")
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    import ctypes
+    lib = cr.lib()
+    st = lib.convrot_int8_linear(ctypes.c_void_p(X.data_ptr()), ctypes.c_void_p(s.data_ptr()),
+                                 ctypes.c_void_p(W.data_ptr()), ctypes.c_void_p(s.data_ptr()),
+                                 M, N, K, ctypes.c_void_p(Y.data_ptr()), None, 0, None)
+    assert st == 7

@@ -1,0 +1,502 @@
+// libconvrot.so: the C ABI declared in include/convrot.h.
+//
+// Host side only: argument validation, TMA tensor-map encoding, launch
+// configuration and the work schedule of the GEMM.  All arithmetic of the
+// method runs in the kernels of rowquant.cuh and gemm.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/convrot.h"
+#include "gemm.cuh"
+#include "rowquant.cuh"
+
+using namespace convrot;
+
+namespace {
+
+// ------------------------------------------------------------------ helpers
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaStream_t as_cuda(convrot_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+struct DeviceInfo {
+  int device = -1;
+  int sms = 0;
+};
+
+DeviceInfo current_device() {
+  static std::mutex mu;
+  static int cached_sms[64] = {0};
+  DeviceInfo d;
+  if (cudaGetDevice(&d.device) != cudaSuccess || d.device < 0 || d.device >= 64) {
+    d.device = -1;
+    return d;
+  }
+  std::lock_guard<std::mutex> g(mu);
+  if (cached_sms[d.device] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d.device) != cudaSuccess) v = 0;
+    cached_sms[d.device] = v;
+  }
+  d.sms = cached_sms[d.device];
+  return d;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor [rows, row_bytes] (row stride = row_bytes), box
+// [box_rows, box_bytes], with or without the 128-byte swizzle.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes,
+                 uint32_t box_rows, uint32_t box_bytes, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE,
+         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+convrot_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ rowquant
+struct RowPlan {
+  int team, rows_per_cta, passes;
+  bool resident;
+};
+
+RowPlan plan_rows(int K) {
+  const int groups = (K + 255) / 256;
+  const int lanes = 4 * groups;  // four threads per virtual 256-group
+  RowPlan p;
+  if (lanes <= 32) {
+    int t = 4;
+    while (t < lanes) t <<= 1;
+    p.team = t;
+    p.passes = 1;
+  } else if (lanes <= 256) {
+    p.team = (lanes + 31) / 32 * 32;
+    p.passes = 1;
+  } else {
+    p.team = 256;
+    p.passes = (lanes + 255) / 256;
+  }
+  p.rows_per_cta = std::max(1, 256 / p.team);
+  p.resident = p.passes == 1;
+  return p;
+}
+
+template <bool ROT, int PRE, int QK, bool RES>
+convrot_status launch_rowquant_t(const RowQuantArgs& a, int threads, cudaStream_t st) {
+  auto k = rowquant_kernel<ROT, PRE, QK, RES>;
+  const DeviceInfo d = current_device();
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, 0) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  const int row_blocks = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
+  const int grid = std::max(1, std::min(row_blocks, std::max(1, per_sm) * std::max(1, d.sms)));
+  k<<<grid, threads, 0, st>>>(a);
+  return launch_status();
+}
+
+template <int PRE, int QK>
+convrot_status launch_rowquant_pre(RowQuantArgs& a, bool rot, cudaStream_t st) {
+  const RowPlan p = plan_rows(a.K);
+  a.team = p.team;
+  a.rows_per_cta = p.rows_per_cta;
+  a.passes = p.passes;
+  const int threads = p.team * p.rows_per_cta;
+  if (rot) {
+    return p.resident ? launch_rowquant_t<true, PRE, QK, true>(a, threads, st)
+                      : launch_rowquant_t<true, PRE, QK, false>(a, threads, st);
+  }
+  return p.resident ? launch_rowquant_t<false, PRE, QK, true>(a, threads, st)
+                    : launch_rowquant_t<false, PRE, QK, false>(a, threads, st);
+}
+
+convrot_status check_group(int group, int K, int multiple) {
+  if (group != 0 && group != 256) return CONVROT_ERR_UNSUPPORTED;
+  if (K <= 0 || K > CONVROT_MAX_K) return CONVROT_ERR_SHAPE;
+  if (K % multiple) return CONVROT_ERR_SHAPE;
+  if (group == 256 && K % 256) return CONVROT_ERR_SHAPE;
+  return CONVROT_OK;
+}
+
+// ------------------------------------------------------------------ GEMM plan
+struct GemmPlan {
+  bool swap;
+  int bn;
+  int tilesA, tilesB, num_tiles, num_kb;
+  int grid;
+  int dp_tiles, sk_iters, sk_q, sk_r;
+  size_t ws_slot_bytes, ws_count_bytes;
+};
+
+int pick_bn_swap(int M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+GemmPlan plan_gemm(int M, int N, int K, int sms) {
+  GemmPlan p{};
+  p.swap = M <= 128;
+  p.bn = p.swap ? pick_bn_swap(M) : 256;
+  const int rowsA = p.swap ? N : M;
+  const int rowsB = p.swap ? M : N;
+  p.tilesA = (rowsA + GEMM_BM - 1) / GEMM_BM;
+  p.tilesB = (rowsB + p.bn - 1) / p.bn;
+  p.num_tiles = p.tilesA * p.tilesB;
+  p.num_kb = (K + GEMM_BK - 1) / GEMM_BK;
+  const long long total = static_cast<long long>(p.num_tiles) * p.num_kb;
+  p.grid = static_cast<int>(std::min<long long>(std::max(1, sms), total));
+  const int waves = p.num_tiles / p.grid;
+  p.dp_tiles = waves >= 2 ? (waves - 1) * p.grid : 0;
+  const int sk_tiles = p.num_tiles - p.dp_tiles;
+  p.sk_iters = sk_tiles * p.num_kb;
+  p.sk_q = p.sk_iters / p.grid;
+  p.sk_r = p.sk_iters % p.grid;
+  // a stream-K region whose iterations split evenly into whole tiles needs no workspace
+  const bool whole = p.sk_r == 0 && p.sk_q % p.num_kb == 0;
+  p.ws_slot_bytes = whole ? 0 : static_cast<size_t>(2) * p.grid * GEMM_BM * p.bn * 4;
+  p.ws_count_bytes = whole ? 0 : static_cast<size_t>(sk_tiles) * 4;
+  return p;
+}
+
+size_t ws_bytes(const GemmPlan& p) {
+  if (p.ws_slot_bytes == 0) return 0;
+  return p.ws_slot_bytes + ((p.ws_count_bytes + 255) / 256) * 256;
+}
+
+template <int BN, bool SWAP, bool W4, int EPI>
+convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs a, int grid,
+                             cudaStream_t st) {
+  using SM = GemmSmem<BN, W4, SWAP>;
+  auto k = gemm_kernel<BN, SWAP, W4, EPI>;
+  // at least ~116 KB so that a second CTA never shares the SM's TMEM
+  const int budget = 200 * 1024;
+  int stages = std::min(GEMM_MAX_STAGES, budget / SM::STAGE);
+  stages = std::max(2, stages);
+  a.stages = stages;
+  const int smem = std::max(SM::total(stages) + 1024, 116 * 1024);
+  static int configured_device_mask = 0;  // per instantiation
+  const DeviceInfo d = current_device();
+  const int bit = 1 << (d.device & 31);
+  if (!(configured_device_mask & bit)) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return CONVROT_ERR_CUDA;
+    configured_device_mask |= bit;
+  }
+  constexpr int threads = W4 ? 320 : 192;
+  k<<<grid, threads, smem, st>>>(ma, mb, a);
+  return launch_status();
+}
+
+template <bool SWAP, bool W4, int EPI>
+convrot_status launch_gemm_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb,
+                              const GemmArgs& a, int grid, cudaStream_t st) {
+  if (!SWAP) return launch_gemm_t<256, false, W4, EPI>(ma, mb, a, grid, st);
+  switch (bn) {
+    case 16: return launch_gemm_t<16, true, W4, EPI>(ma, mb, a, grid, st);
+    case 32: return launch_gemm_t<32, true, W4, EPI>(ma, mb, a, grid, st);
+    case 64: return launch_gemm_t<64, true, W4, EPI>(ma, mb, a, grid, st);
+    default: return launch_gemm_t<128, true, W4, EPI>(ma, mb, a, grid, st);
+  }
+}
+
+convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* s_tok,
+                        const float* s_row, int M, int N, int K, void* out, bool s32_out,
+                        void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
+  const GemmPlan p = plan_gemm(M, N, K, d.sms);
+  const size_t need = ws_bytes(p);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CONVROT_ERR_WORKSPACE;
+  if (need > 0 && !aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
+
+  const int bn = p.bn;
+  CUtensorMap mx, mw;
+  // activations: int8 [M, K]; weights: int8 [N, K] or packed [N, K/2]
+  const uint32_t x_box_rows = p.swap ? bn : GEMM_BM;
+  const uint32_t w_box_rows = p.swap ? GEMM_BM : bn;
+  if (!make_map_u8(&mx, Xq, M, K, x_box_rows, GEMM_BK, true)) return CONVROT_ERR_CUDA;
+  if (w4) {
+    if (!make_map_u8(&mw, Wq, N, K / 2, w_box_rows, GEMM_BK / 2, false)) return CONVROT_ERR_CUDA;
+  } else {
+    if (!make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK, true)) return CONVROT_ERR_CUDA;
+  }
+
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.rowsA = p.swap ? N : M;
+  a.rowsB = p.swap ? M : N;
+  a.tilesA = p.tilesA;
+  a.tilesB = p.tilesB;
+  a.num_tiles = p.num_tiles;
+  a.num_kb = p.num_kb;
+  a.dp_tiles = p.dp_tiles;
+  a.sk_iters = p.sk_iters;
+  a.sk_q = p.sk_q;
+  a.sk_r = p.sk_r;
+  a.s_tok = s_tok;
+  a.s_row = s_row;
+  a.out = out;
+  a.ws_slots = need ? static_cast<int32_t*>(workspace) : nullptr;
+  a.ws_counts = need ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + p.ws_slot_bytes)
+                     : nullptr;
+  const CUtensorMap& ma = p.swap ? mw : mx;
+  const CUtensorMap& mb = p.swap ? mx : mw;
+  if (w4) {
+    if (s32_out)
+      return p.swap ? launch_gemm_bn<true, true, EPI_S32>(bn, ma, mb, a, p.grid, st)
+                    : launch_gemm_bn<false, true, EPI_S32>(bn, ma, mb, a, p.grid, st);
+    return p.swap ? launch_gemm_bn<true, true, EPI_BF16>(bn, ma, mb, a, p.grid, st)
+                  : launch_gemm_bn<false, true, EPI_BF16>(bn, ma, mb, a, p.grid, st);
+  }
+  if (s32_out)
+    return p.swap ? launch_gemm_bn<true, false, EPI_S32>(bn, ma, mb, a, p.grid, st)
+                  : launch_gemm_bn<false, false, EPI_S32>(bn, ma, mb, a, p.grid, st);
+  return p.swap ? launch_gemm_bn<true, false, EPI_BF16>(bn, ma, mb, a, p.grid, st)
+                : launch_gemm_bn<false, false, EPI_BF16>(bn, ma, mb, a, p.grid, st);
+}
+
+convrot_status check_gemm_shape(int M, int N, int K, bool w4) {
+  if (M < 0 || N < 0 || K <= 0 || K > CONVROT_MAX_K) return CONVROT_ERR_SHAPE;
+  if (K % (w4 ? 32 : 16)) return CONVROT_ERR_SHAPE;
+  if (N % 8) return CONVROT_ERR_SHAPE;
+  return CONVROT_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int convrot_version(void) { return (1 << 16) | 0; }
+
+const char* convrot_status_string(convrot_status st) {
+  switch (st) {
+    case CONVROT_OK: return "CONVROT_OK";
+    case CONVROT_ERR_NULL: return "CONVROT_ERR_NULL: a required pointer is NULL";
+    case CONVROT_ERR_SHAPE: return "CONVROT_ERR_SHAPE: unsupported or inconsistent size";
+    case CONVROT_ERR_ALIGN: return "CONVROT_ERR_ALIGN: pointer not aligned as required";
+    case CONVROT_ERR_UNSUPPORTED: return "CONVROT_ERR_UNSUPPORTED: unsupported option";
+    case CONVROT_ERR_CUDA: return "CONVROT_ERR_CUDA: a CUDA call failed";
+    case CONVROT_ERR_DEVICE_TIMEOUT: return "CONVROT_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    case CONVROT_ERR_WORKSPACE: return "CONVROT_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "CONVROT_ERR_UNKNOWN";
+}
+
+convrot_status convrot_device_status(convrot_stream_t stream, uint32_t* detail) {
+  if (cudaStreamSynchronize(as_cuda(stream)) != cudaSuccess) return CONVROT_ERR_CUDA;
+  unsigned v = 0;
+  const unsigned zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(v)) != cudaSuccess) return CONVROT_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  if (detail) *detail = v;
+  return v ? CONVROT_ERR_DEVICE_TIMEOUT : CONVROT_OK;
+}
+
+convrot_status convrot_quantize_weight(const void* W, int N, int K, int group,
+                                       const float* col_scale, int8_t* Wq, float* s_row,
+                                       convrot_stream_t stream) {
+  if (N < 0) return CONVROT_ERR_SHAPE;
+  const convrot_status g = check_group(group, K, 16);
+  if (g != CONVROT_OK) return g;
+  if (N == 0) return CONVROT_OK;
+  if (!W || !Wq || !s_row) return CONVROT_ERR_NULL;
+  if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(s_row, 4)) return CONVROT_ERR_ALIGN;
+  if (col_scale && !aligned(col_scale, 16)) return CONVROT_ERR_ALIGN;
+  RowQuantArgs a{};
+  a.src = static_cast<const uint16_t*>(W);
+  a.vec = col_scale;
+  a.dst8 = Wq;
+  a.scale = s_row;
+  a.rows = N;
+  a.K = K;
+  const bool rot = group == 256;
+  return col_scale ? launch_rowquant_pre<PRE_COLSCALE, QK_INT8>(a, rot, as_cuda(stream))
+                   : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, rot, as_cuda(stream));
+}
+
+convrot_status convrot_quantize_weight_w4(const void* W, int N, int K, int group,
+                                          const float* col_scale, float clip_lo,
+                                          float clip_hi, int clip_steps, uint8_t* Wq4,
+                                          float* s_row, convrot_stream_t stream) {
+  if (N < 0) return CONVROT_ERR_SHAPE;
+  const convrot_status g = check_group(group, K, 32);
+  if (g != CONVROT_OK) return g;
+  if (clip_steps < 1 || clip_steps > 64 || !(clip_lo > 0.f) || !(clip_hi >= clip_lo))
+    return CONVROT_ERR_SHAPE;
+  if (N == 0) return CONVROT_OK;
+  if (!W || !Wq4 || !s_row) return CONVROT_ERR_NULL;
+  if (!aligned(W, 16) || !aligned(Wq4, 16) || !aligned(s_row, 4)) return CONVROT_ERR_ALIGN;
+  if (col_scale && !aligned(col_scale, 16)) return CONVROT_ERR_ALIGN;
+  RowQuantArgs a{};
+  a.src = static_cast<const uint16_t*>(W);
+  a.vec = col_scale;
+  a.dst4 = Wq4;
+  a.scale = s_row;
+  a.rows = N;
+  a.K = K;
+  if (clip_steps == 1) {
+    a.clip_lo = clip_hi;
+    a.clip_step = 0.f;
+  } else {
+    a.clip_lo = clip_lo;
+    a.clip_step = static_cast<float>((static_cast<double>(clip_hi) - clip_lo) / (clip_steps - 1));
+  }
+  a.clip_steps = clip_steps;
+  const bool rot = group == 256;
+  return col_scale ? launch_rowquant_pre<PRE_COLSCALE, QK_INT4>(a, rot, as_cuda(stream))
+                   : launch_rowquant_pre<PRE_NONE, QK_INT4>(a, rot, as_cuda(stream));
+}
+
+convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
+                                        const float* norm_w, float eps, int8_t* Xq,
+                                        float* s_tok, convrot_stream_t stream) {
+  if (M < 0) return CONVROT_ERR_SHAPE;
+  const convrot_status g = check_group(group, K, 16);
+  if (g != CONVROT_OK) return g;
+  if (norm_w && !(eps >= 0.f)) return CONVROT_ERR_SHAPE;
+  if (M == 0) return CONVROT_OK;
+  if (!x || !Xq || !s_tok) return CONVROT_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(Xq, 16) || !aligned(s_tok, 4)) return CONVROT_ERR_ALIGN;
+  if (norm_w && !aligned(norm_w, 16)) return CONVROT_ERR_ALIGN;
+  RowQuantArgs a{};
+  a.src = static_cast<const uint16_t*>(x);
+  a.vec = norm_w;
+  a.dst8 = Xq;
+  a.scale = s_tok;
+  a.rows = M;
+  a.K = K;
+  a.eps = eps;
+  const bool rot = group == 256;
+  return norm_w ? launch_rowquant_pre<PRE_NORM, QK_INT8>(a, rot, as_cuda(stream))
+                : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, rot, as_cuda(stream));
+}
+
+convrot_status convrot_smoothquant_calibrate(const void* x, int M, int K, const float* norm_w,
+                                             float eps, const void* W, int N, float alpha,
+                                             float* smooth, float* norm_w_folded,
+                                             convrot_stream_t stream) {
+  if (M <= 0 || N <= 0 || K <= 0 || K > CONVROT_MAX_K || K % 16) return CONVROT_ERR_SHAPE;
+  if (!(alpha >= 0.f && alpha <= 1.f) || !(eps >= 0.f)) return CONVROT_ERR_SHAPE;
+  if (!x || !norm_w || !W || !smooth || !norm_w_folded) return CONVROT_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(W, 16) || !aligned(norm_w, 4) || !aligned(smooth, 4) ||
+      !aligned(norm_w_folded, 4))
+    return CONVROT_ERR_ALIGN;
+  if (norm_w_folded == norm_w) return CONVROT_ERR_UNSUPPORTED;
+  cudaStream_t st = as_cuda(stream);
+  if (cudaMemsetAsync(smooth, 0, sizeof(float) * K, st) != cudaSuccess) return CONVROT_ERR_CUDA;
+  if (cudaMemsetAsync(norm_w_folded, 0, sizeof(float) * K, st) != cudaSuccess)
+    return CONVROT_ERR_CUDA;
+  calib_act_colmax<<<(M + CAL_ROWS - 1) / CAL_ROWS, 256, 0, st>>>(
+      static_cast<const uint16_t*>(x), M, K, norm_w, eps, reinterpret_cast<unsigned*>(smooth));
+  calib_weight_colmax<<<(N + CAL_ROWS - 1) / CAL_ROWS, 256, 0, st>>>(
+      static_cast<const uint16_t*>(W), N, K, reinterpret_cast<unsigned*>(norm_w_folded));
+  calib_finalize<<<(K + 255) / 256, 256, 0, st>>>(norm_w, K, alpha, smooth, norm_w_folded);
+  return launch_status();
+}
+
+size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits) {
+  if (check_gemm_shape(M, N, K, weight_bits == 4) != CONVROT_OK) return 0;
+  if (weight_bits != 8 && weight_bits != 4) return 0;
+  if (M == 0 || N == 0) return 0;
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return 0;
+  return ws_bytes(plan_gemm(M, N, K, d.sms));
+}
+
+static convrot_status linear_common(const int8_t* Xq, const float* s_tok, const void* Wq,
+                                    bool w4, const float* s_row, int M, int N, int K, void* Y,
+                                    void* workspace, size_t workspace_bytes,
+                                    convrot_stream_t stream) {
+  const convrot_status sh = check_gemm_shape(M, N, K, w4);
+  if (sh != CONVROT_OK) return sh;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  if (!Xq || !s_tok || !Wq || !s_row || !Y) return CONVROT_ERR_NULL;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(s_tok, 4) ||
+      !aligned(s_row, 4))
+    return CONVROT_ERR_ALIGN;
+  return run_gemm(Xq, Wq, w4, s_tok, s_row, M, N, K, Y, false, workspace, workspace_bytes,
+                  as_cuda(stream));
+}
+
+convrot_status convrot_int8_linear(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
+                                   const float* s_row, int M, int N, int K, void* Y,
+                                   void* workspace, size_t workspace_bytes,
+                                   convrot_stream_t stream) {
+  return linear_common(Xq, s_tok, Wq, false, s_row, M, N, K, Y, workspace, workspace_bytes,
+                       stream);
+}
+
+convrot_status convrot_w4a8_linear(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
+                                   const float* s_row, int M, int N, int K, void* Y,
+                                   void* workspace, size_t workspace_bytes,
+                                   convrot_stream_t stream) {
+  return linear_common(Xq, s_tok, Wq4, true, s_row, M, N, K, Y, workspace, workspace_bytes,
+                       stream);
+}
+
+// The raw-accumulator entry points run the same kernels and schedule with
+// the int32 epilogue.
+static convrot_status gemm_s32_common(const int8_t* Xq, const void* Wq, bool w4, int M, int N,
+                                      int K, int32_t* acc, void* workspace,
+                                      size_t workspace_bytes, convrot_stream_t stream) {
+  const convrot_status sh = check_gemm_shape(M, N, K, w4);
+  if (sh != CONVROT_OK) return sh;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  if (!Xq || !Wq || !acc) return CONVROT_ERR_NULL;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(acc, 16)) return CONVROT_ERR_ALIGN;
+  return run_gemm(Xq, Wq, w4, nullptr, nullptr, M, N, K, acc, true, workspace, workspace_bytes,
+                  as_cuda(stream));
+}
+
+convrot_status convrot_int8_gemm_s32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
+                                     int32_t* acc, void* workspace, size_t workspace_bytes,
+                                     convrot_stream_t stream) {
+  return gemm_s32_common(Xq, Wq, false, M, N, K, acc, workspace, workspace_bytes, stream);
+}
+
+convrot_status convrot_w4a8_gemm_s32(const int8_t* Xq, const uint8_t* Wq4, int M, int N, int K,
+                                     int32_t* acc, void* workspace, size_t workspace_bytes,
+                                     convrot_stream_t stream) {
+  return gemm_s32_common(Xq, Wq4, true, M, N, K, acc, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"

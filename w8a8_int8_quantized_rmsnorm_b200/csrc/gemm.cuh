@@ -1,0 +1,525 @@
+// W8A8 / W4A8 ConvRot linear on the 5th-generation tensor core.
+//
+//   acc[m, n] = sum_k Xq[m, k] * Wq[n, k]                 (exact int32)
+//   Y[m, n]   = bf16_rn(float(acc) * s_tok[m] * s_row[n])
+//
+// ("MOSS-Image Qwen3.5-9B text encoder, INT8 (W8A8, ConvRot)", file table,
+// "Matmul" row; the int4 weight layout of "MossInt4", "Format".)
+//
+// Kernel structure (one CTA per SM, persistent):
+//   warp 0      TMA producer: int8 tiles of both operands, 128 bytes of K per
+//               stage, 128-byte swizzle, into a ring of shared-memory stages;
+//   warp 1      allocates TMEM and issues tcgen05.mma kind::i8 (one thread),
+//               128 x BN x 32 per instruction, s32 accumulators in TMEM,
+//               two accumulator buffers so the epilogue of one tile overlaps
+//               the main loop of the next;
+//   warps 2-5   epilogue: tcgen05.ld of the accumulators, dequantisation to
+//               bf16 (or raw int32), global stores;
+//   warps 6-9   (int4 weights only) unpack two signed nibbles per byte into
+//               the swizzled int8 stage the MMA reads.  A nibble n is written
+//               as the byte n * 16 (the nibble in the high half), so the MMA
+//               accumulates 16 * acc exactly and the epilogue divides by 16.
+//
+// Operand roles.  Operand A fills the MMA's M = 128 rows, operand B its N = BN
+// columns.  For M > 128 tokens A = activations and B = weights (BN = 256).
+// For M <= 128 the roles swap (A = weights, B = tokens, BN = 16..128), so the
+// 128-row tensor-core dimension is filled by weight rows and every weight
+// byte is streamed exactly once.
+//
+// Work split.  Output tiles are ordered in groups of 8 A-tiles for L2 reuse.
+// Whole waves of tiles are handed out round-robin (data-parallel).  The last
+// one to two waves are split evenly by K-block over all CTAs (stream-K).  A
+// CTA whose range covers only part of a tile writes its int32 partial tile to
+// its own workspace slot, then increments the tile's counter; the CTA that
+// brings the counter to the number of contributors sums all partial slots in
+// a fixed order (deterministic), writes the output and resets the counter.
+// No CTA ever waits on another CTA.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace convrot {
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BK = 128;  // int8 elements (bytes) of K per stage
+constexpr int GEMM_UMMA_K = 32;
+constexpr int GEMM_MAX_STAGES = 16;
+constexpr int GEMM_GROUP_A = 8;
+constexpr int EPI_BF16 = 0;
+constexpr int EPI_S32 = 1;
+
+// wait sites recorded in the device error word
+constexpr unsigned SITE_PROD_EMPTY = 1, SITE_MMA_FULL = 2, SITE_MMA_TMEM = 3, SITE_EPI_FULL = 4,
+                   SITE_CONV_FULL = 5, SITE_DRAIN = 6, SITE_EPI_SYNC = 7;
+
+struct GemmArgs {
+  int M, N, K;
+  int rowsA, rowsB;  // rows of operands A and B
+  int tilesA, tilesB;
+  int num_tiles;
+  int num_kb;
+  int stages;
+  int dp_tiles;      // tiles [0, dp_tiles) are data-parallel
+  int sk_iters;      // (num_tiles - dp_tiles) * num_kb
+  int sk_q, sk_r;    // stream-K split: first sk_r CTAs get sk_q + 1 iterations
+  const float* s_tok;
+  const float* s_row;
+  void* out;
+  int32_t* ws_slots;     // [2 * gridDim.x][BM * BN] partial tiles
+  unsigned* ws_counts;   // [num_tiles - dp_tiles]
+};
+
+struct Segment {
+  int tile, kb0, kb1;
+  bool partial;
+  int slot;
+};
+
+struct Schedule {
+  const GemmArgs* p;
+  int cta, ncta;
+  int dp_next;
+  int sk_begin, sk_end, sk_cur;
+
+  __device__ void init(const GemmArgs& a) {
+    p = &a;
+    cta = blockIdx.x;
+    ncta = gridDim.x;
+    dp_next = cta;
+    sk_begin = cta * a.sk_q + min(cta, a.sk_r);
+    sk_end = sk_begin + a.sk_q + (cta < a.sk_r ? 1 : 0);
+    sk_cur = sk_begin;
+  }
+  __device__ bool next(Segment& s) {
+    if (dp_next < p->dp_tiles) {
+      s.tile = dp_next;
+      s.kb0 = 0;
+      s.kb1 = p->num_kb;
+      s.partial = false;
+      s.slot = -1;
+      dp_next += ncta;
+      return true;
+    }
+    if (sk_cur < sk_end) {
+      const int u = sk_cur / p->num_kb;
+      s.kb0 = sk_cur - u * p->num_kb;
+      s.kb1 = min(p->num_kb, s.kb0 + (sk_end - sk_cur));
+      s.tile = p->dp_tiles + u;
+      s.partial = !(s.kb0 == 0 && s.kb1 == p->num_kb);
+      s.slot = 2 * cta + (sk_cur == sk_begin ? 0 : 1);
+      sk_cur += s.kb1 - s.kb0;
+      return true;
+    }
+    return false;
+  }
+};
+
+// CTA that owns stream-K iteration i.
+__device__ __forceinline__ int sk_owner(const GemmArgs& a, int i) {
+  const int big = a.sk_r * (a.sk_q + 1);
+  if (i < big) return i / (a.sk_q + 1);
+  return a.sk_r + (i - big) / a.sk_q;
+}
+__device__ __forceinline__ int sk_begin_of(const GemmArgs& a, int c) {
+  return c * a.sk_q + min(c, a.sk_r);
+}
+
+__device__ __forceinline__ void tile_coords(const GemmArgs& a, int tile, int& ta, int& tb) {
+  const int per_group = GEMM_GROUP_A * a.tilesB;
+  const int group = tile / per_group;
+  const int first = group * GEMM_GROUP_A;
+  const int ga = min(GEMM_GROUP_A, a.tilesA - first);
+  const int local = tile - group * per_group;
+  ta = first + local % ga;
+  tb = local / ga;
+}
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Shared-memory plan (offsets from a 1024-byte aligned base).
+template <int BN, bool W4, bool SWAP>
+struct GemmSmem {
+  static constexpr int A_BYTES = GEMM_BM * GEMM_BK;
+  static constexpr int B_BYTES = BN * GEMM_BK;
+  static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
+  static constexpr int P_BYTES = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 weight tile
+  static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;  // TMEM columns per accumulator buffer
+  static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
+  static constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
+  __host__ __device__ static int bar_offset(int stages) { return stages * STAGE; }
+  // full, empty, conv: stages each; tmem_full, tmem_empty: 2 each; + scalars
+  __host__ __device__ static int total(int stages) {
+    return bar_offset(stages) + (3 * GEMM_MAX_STAGES + 6) * 8 + 64;
+  }
+};
+
+template <int BN, bool SWAP, bool W4, int EPI>
+__global__ void __launch_bounds__(W4 ? 320 : 192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                GemmArgs a) {
+  using SM = GemmSmem<BN, W4, SWAP>;
+  constexpr int CW = SM::CW;
+  constexpr uint32_t IDESC = idesc_s8s8s32(GEMM_BM, BN);
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int S = a.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::bar_offset(S));
+  uint64_t* empty = full + GEMM_MAX_STAGES;
+  uint64_t* conv = empty + GEMM_MAX_STAGES;
+  uint64_t* tmem_full = conv + GEMM_MAX_STAGES;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* drain = tmem_empty + 2;
+  uint64_t* epi_sync = drain + 1;  // rendezvous of the four epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&conv[s], 128);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    mbar_init(epi_sync, 4);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, SM::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  Schedule sched;
+  sched.init(a);
+  Segment seg;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_last();
+      const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_first();
+      uint32_t tx = 0;
+      if (W4) {
+        tx = SWAP ? (SM::P_BYTES + SM::B_BYTES) : (SM::A_BYTES + SM::P_BYTES);
+      } else {
+        tx = SM::A_BYTES + SM::B_BYTES;
+      }
+      uint32_t it = 0;
+      bool ok = true;
+      while (ok && sched.next(seg)) {
+        int ta, tb;
+        tile_coords(a, seg.tile, ta, tb);
+        for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, SITE_PROD_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * SM::STAGE;
+          mbar_arrive_expect_tx(&full[s], tx);
+          if (W4 && SWAP)
+            tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmA, &full[s], kb * (GEMM_BK / 2),
+                        ta * GEMM_BM, pol_a);
+          else
+            tma_load_2d(st, &tmA, &full[s], kb * GEMM_BK, ta * GEMM_BM, pol_a);
+          if (W4 && !SWAP)
+            tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], kb * (GEMM_BK / 2),
+                        tb * BN, pol_b);
+          else
+            tma_load_2d(st + SM::A_BYTES, &tmB, &full[s], kb * GEMM_BK, tb * BN, pol_b);
+        }
+      }
+      // drain: make sure no copy is still landing in shared memory when the CTA exits
+      const uint32_t n_issued = it;
+      const uint32_t first = n_issued > static_cast<uint32_t>(S) ? n_issued - S : 0u;
+      for (uint32_t j = first; j < n_issued; ++j) {
+        int dummy = 0;
+        volatile int* never = &dummy;
+        mbar_wait(&full[j % S], (j / S) & 1u, never, SITE_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      while (ok && sched.next(seg)) {
+        const uint32_t b = local & 1u;
+        const uint32_t use = local >> 1;
+        if (!mbar_wait(&tmem_empty[b], (use & 1u) ^ 1u, abort_flag, SITE_MMA_TMEM)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + b * SM::ACC_STRIDE;
+        for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(W4 ? &conv[s] : &full[s], ph, abort_flag, SITE_MMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(smem + s * SM::STAGE);
+          const uint32_t sb = sa + SM::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
+            mma_s8(d, sw128_kmajor_desc(sa + k * GEMM_UMMA_K), sw128_kmajor_desc(sb + k * GEMM_UMMA_K),
+                   IDESC, (kb > seg.kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&tmem_full[b]);
+        ++local;
+      }
+      // every MMA this thread issued must be complete before TMEM is released
+      mma_commit(drain);
+      int never = 0;
+      mbar_wait(drain, 0u, &never, SITE_DRAIN);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int et = threadIdx.x - 64;  // 0..127 within the epilogue group
+    uint32_t local = 0;
+    uint32_t sync_phase = 0;
+    // bounded rendezvous of the four epilogue warps (never an unbounded bar.sync)
+    auto epi_rendezvous = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_sync);
+      const bool r = mbar_wait(epi_sync, sync_phase & 1u, abort_flag, SITE_EPI_SYNC);
+      ++sync_phase;
+      __syncwarp();
+      return r;
+    };
+    while (sched.next(seg)) {
+      const uint32_t b = local & 1u;
+      const uint32_t use = local >> 1;
+      const bool got = mbar_wait(&tmem_full[b], use & 1u, abort_flag, SITE_EPI_FULL);
+      __syncwarp();
+      if (!got) break;
+      tc_fence_after();
+      int ta, tb;
+      tile_coords(a, seg.tile, ta, tb);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * SM::ACC_STRIDE;
+      const int arow = ta * GEMM_BM + 32 * q + lane;  // operand-A row of this thread
+
+      if (seg.partial) {
+        // write this CTA's partial tile to its slot
+        int32_t* slot = a.ws_slots + static_cast<size_t>(seg.slot) * (GEMM_BM * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / CW; ++c) {
+          uint32_t r[32];
+          if (CW == 32) {
+            tmem_ld_32x32b_x32(tbase + c * CW, r);
+          } else {
+            tmem_ld_32x32b_x16(tbase + c * CW, r);
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int j4 = 0; j4 < CW / 4; ++j4) {
+            uint4* dst = reinterpret_cast<uint4*>(slot) + ((c * 4 + q) * (CW / 4) + j4) * 32 + lane;
+            *dst = make_uint4(r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+          }
+        }
+      }
+      // the accumulator buffer can be reused once a partial tile is saved
+      // (a full tile keeps it until its output is written, below)
+      bool finalize = !seg.partial;
+      if (seg.partial) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tmem_empty[b]);
+        __threadfence();
+        if (!epi_rendezvous()) break;
+        if (et == 0) {
+          const int u = seg.tile - a.dp_tiles;
+          const int c_lo = sk_owner(a, u * a.num_kb);
+          const int c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
+          const unsigned prev = atomicAdd(&a.ws_counts[u], 1u);
+          const bool last = prev + 1u == static_cast<unsigned>(c_hi - c_lo + 1);
+          if (last) a.ws_counts[u] = 0u;  // leave the workspace clean for the next call
+          *last_flag = last ? 1 : 0;
+        }
+        if (!epi_rendezvous()) break;
+        finalize = *last_flag != 0;
+        if (finalize) __threadfence();
+      }
+      if (finalize) {
+        int c_lo = 0, c_hi = -1, u = 0;
+        if (seg.partial) {
+          u = seg.tile - a.dp_tiles;
+          c_lo = sk_owner(a, u * a.num_kb);
+          c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / CW; ++c) {
+          uint32_t r[32];
+          if (!seg.partial) {
+            if (CW == 32) {
+              tmem_ld_32x32b_x32(tbase + c * CW, r);
+            } else {
+              tmem_ld_32x32b_x16(tbase + c * CW, r);
+            }
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < CW; ++j) r[j] = 0u;
+            for (int cc = c_lo; cc <= c_hi; ++cc) {
+              const int slot_id = 2 * cc + (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
+              const uint4* src = reinterpret_cast<const uint4*>(
+                                     a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN)) +
+                                 (c * 4 + q) * (CW / 4) * 32 + lane;
+#pragma unroll
+              for (int j4 = 0; j4 < CW / 4; ++j4) {
+                const uint4 v = __ldcg(src + j4 * 32);
+                r[4 * j4] += v.x;
+                r[4 * j4 + 1] += v.y;
+                r[4 * j4 + 2] += v.z;
+                r[4 * j4 + 3] += v.w;
+              }
+            }
+          }
+          // ---- store one CW-column chunk
+          if (!SWAP) {
+            const int m = arow;
+            const int n0 = tb * BN + c * CW;
+            if (m < a.M) {
+              if (EPI == EPI_BF16) {
+                const float st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
+                __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(m) * a.N;
+#pragma unroll
+                for (int j8 = 0; j8 < CW / 8; ++j8) {
+                  const int n = n0 + 8 * j8;
+                  if (n < a.N) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                      const float y0 = static_cast<float>(static_cast<int32_t>(r[8 * j8 + 2 * h])) * st * __ldg(a.s_row + n + 2 * h);
+                      const float y1 = static_cast<float>(static_cast<int32_t>(r[8 * j8 + 2 * h + 1])) * st * __ldg(a.s_row + n + 2 * h + 1);
+                      w[h] = pack_bf16x2(y0, y1);
+                    }
+                    *reinterpret_cast<uint4*>(y + n) = make_uint4(w[0], w[1], w[2], w[3]);
+                  }
+                }
+              } else {
+                int32_t* y = reinterpret_cast<int32_t*>(a.out) + static_cast<size_t>(m) * a.N;
+#pragma unroll
+                for (int j4 = 0; j4 < CW / 4; ++j4) {
+                  const int n = n0 + 4 * j4;
+                  if (n < a.N) {
+                    const int sh = W4 ? 4 : 0;
+                    *reinterpret_cast<int4*>(y + n) =
+                        make_int4(static_cast<int32_t>(r[4 * j4]) >> sh, static_cast<int32_t>(r[4 * j4 + 1]) >> sh,
+                                  static_cast<int32_t>(r[4 * j4 + 2]) >> sh, static_cast<int32_t>(r[4 * j4 + 3]) >> sh);
+                  }
+                }
+              }
+            }
+          } else {
+            const int n = arow;  // weight row
+            const int m0 = tb * BN + c * CW;
+            if (n < a.N) {
+              if (EPI == EPI_BF16) {
+                const float sr = a.s_row[n] * (W4 ? 0.0625f : 1.0f);
+                __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.out);
+#pragma unroll
+                for (int j = 0; j < CW; ++j) {
+                  const int m = m0 + j;
+                  if (m < a.M) {
+                    const float v = static_cast<float>(static_cast<int32_t>(r[j])) * __ldg(a.s_tok + m) * sr;
+                    y[static_cast<size_t>(m) * a.N + n] = __float2bfloat16_rn(v);
+                  }
+                }
+              } else {
+                int32_t* y = reinterpret_cast<int32_t*>(a.out);
+#pragma unroll
+                for (int j = 0; j < CW; ++j) {
+                  const int m = m0 + j;
+                  if (m < a.M) y[static_cast<size_t>(m) * a.N + n] = static_cast<int32_t>(r[j]) >> (W4 ? 4 : 0);
+                }
+              }
+            }
+          }
+        }
+      }
+      if (!seg.partial) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tmem_empty[b]);
+      }
+      ++local;
+    }
+  } else if (W4) {
+    // ------------------------------------------------------------ int4 unpack
+    const int ct = threadIdx.x - 192;  // 0..127
+    constexpr int WR = SM::W_ROWS;
+    uint32_t it = 0;
+    bool ok = true;
+    while (ok && sched.next(seg)) {
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, SITE_CONV_FULL)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * SM::STAGE;
+        const uint8_t* packed = st + SM::A_BYTES + SM::B_BYTES;
+        uint8_t* unp = SWAP ? st : st + SM::A_BYTES;
+        for (int idx = ct; idx < WR * 4; idx += 128) {
+          const int r = idx >> 2, pc = idx & 3;
+          const uint4 pk = *reinterpret_cast<const uint4*>(packed + r * 64 + pc * 16);
+          const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint32_t lo = (w[h] << 4) & 0xF0F0F0F0u;
+            const uint32_t hi = w[h] & 0xF0F0F0F0u;
+            o[2 * h] = __byte_perm(lo, hi, 0x5140);
+            o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+          }
+          const int sw = r & 7;
+          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&conv[s]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, SM::TMEM_COLS);
+  }
+}
+
+}  // namespace convrot
