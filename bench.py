@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--copies", type=int, default=0,
+                    help="input copies rotated through to defeat L2 (0 = enough for 3x L2)")
     return ap.parse_args()
 
 
@@ -213,6 +215,8 @@ def run_ours(args, rank, world, dev):
     # copies of the per-step operands so that no step finds its inputs in L2
     step_bytes = sum(x.numel() * 2 for x in inputs) + sum(l.Wq.numel() for l in layers)
     copies = 1 if step_bytes > 2 * L2_BYTES else min(8, math.ceil(3 * L2_BYTES / step_bytes))
+    if args.copies > 0:
+        copies = args.copies
     x_sets = [inputs] + [[x.clone() for x in inputs] for _ in range(copies - 1)]
     w_sets = [[(l.Wq, l.s_row) for l in layers]] + \
              [[(l.Wq.clone(), l.s_row.clone()) for l in layers] for _ in range(copies - 1)]

@@ -180,7 +180,9 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits);
  * tiles of output tiles that several CTAs share (scratch) and one arrival
  * counter per such tile; every call that returns CONVROT_OK leaves the
  * counters at zero again, so the buffer can be passed to later calls without
- * clearing.  Calls that share one workspace must not run concurrently.
+ * clearing, also by calls of other shapes (the counters occupy a fixed
+ * region at the start of the buffer).  Calls that share one workspace must
+ * not run concurrently.
  */
 convrot_status convrot_int8_linear(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
                                    const float* s_row, int M, int N, int K, void* Y,

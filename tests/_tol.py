@@ -21,16 +21,20 @@ import numpy as np
 U = 2.0 ** -24
 
 
-def row_error(v, group, pre):
-    """E / absmax per row (0 for all-zero rows), for the rotated values v."""
+def row_error(v, group, pre, extra_rel=0.0):
+    """E / absmax per row (0 for all-zero rows), for the rotated values v.
+
+    extra_rel is an additional relative perturbation of the inputs, e.g. when
+    the two sides derived a per-column multiplier independently."""
     v = np.asarray(v, dtype=np.float64)
     amax = np.max(np.abs(v), axis=1)
+    in_rel = (2.0 * U if pre else 0.0) + extra_rel
     if group:
         M, K = v.shape
         gn = np.sqrt(np.sum(v.reshape(M, K // group, group) ** 2, axis=2)).max(axis=1)
-        E = (8.0 + (2.0 if pre else 0.0)) * U * gn
+        E = (8.0 * U + in_rel) * gn
     else:
-        E = (2.0 * U if pre else 0.0) * amax
+        E = in_rel * amax
     with np.errstate(divide="ignore", invalid="ignore"):
         r = np.where(amax > 0, E / np.where(amax > 0, amax, 1.0), 0.0)
     return r, amax

@@ -128,7 +128,20 @@ def test_workspace_reuse_and_determinism(cr):
         acc = cr.convrot_int8_gemm_s32(Xd, Wd, workspace=ws)
         torch.cuda.synchronize()
         assert np.array_equal(acc.cpu().numpy().astype(np.int64), want)
-    assert int(ws.buf[-256:].count_nonzero().item()) == 0
+    # the counters live in the first 4 KB and are back at zero
+    assert int(ws.buf[:4096].count_nonzero().item()) == 0
+
+
+def test_workspace_shared_across_shapes(cr):
+    # one buffer, calls of different shapes and operand roles in a row
+    ws = cr.Workspace()
+    for (M, N, K) in [(512, 4096, 12288), (1, 24576, 4096), (129, 264, 512), (2048, 1024, 4096),
+                      (16, 1024, 4096), (512, 4096, 12288)]:
+        X = _rand_i8((M, K), M + N)
+        W = _rand_i8((N, K), N + K)
+        acc = cr.convrot_int8_gemm_s32(X.cuda(), W.cuda(), workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref.int_matmul(X.numpy(), W.numpy()))
 
 
 def test_workspace_too_small_is_rejected(cr):

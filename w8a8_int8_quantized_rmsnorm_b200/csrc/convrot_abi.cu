@@ -152,6 +152,8 @@ convrot_status check_group(int group, int K, int multiple) {
 }
 
 // ------------------------------------------------------------------ GEMM plan
+constexpr size_t kCounterBytes = 4096;
+
 struct GemmPlan {
   bool swap;
   int bn;
@@ -179,7 +181,9 @@ GemmPlan plan_gemm(int M, int N, int K, int sms) {
   p.num_tiles = p.tilesA * p.tilesB;
   p.num_kb = (K + GEMM_BK - 1) / GEMM_BK;
   const long long total = static_cast<long long>(p.num_tiles) * p.num_kb;
-  p.grid = static_cast<int>(std::min<long long>(std::max(1, sms), total));
+  // at most 2 * grid tiles are split, so the fixed counter region always fits
+  const int max_grid = static_cast<int>(kCounterBytes / 4 / 2);
+  p.grid = static_cast<int>(std::min<long long>(std::min(std::max(1, sms), max_grid), total));
   const int waves = p.num_tiles / p.grid;
   p.dp_tiles = waves >= 2 ? (waves - 1) * p.grid : 0;
   const int sk_tiles = p.num_tiles - p.dp_tiles;
@@ -193,9 +197,13 @@ GemmPlan plan_gemm(int M, int N, int K, int sms) {
   return p;
 }
 
+// Workspace layout: a fixed region of tile counters at offset 0 (left at zero
+// by every successful call, whatever the shape), then the partial-tile slots.
+// Keeping the counters at a fixed place is what makes one zero-filled buffer
+// reusable across calls of different shapes.
 size_t ws_bytes(const GemmPlan& p) {
   if (p.ws_slot_bytes == 0) return 0;
-  return p.ws_slot_bytes + ((p.ws_count_bytes + 255) / 256) * 256;
+  return kCounterBytes + p.ws_slot_bytes;
 }
 
 template <int BN, bool SWAP, bool W4, int EPI>
@@ -273,9 +281,9 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
   a.s_tok = s_tok;
   a.s_row = s_row;
   a.out = out;
-  a.ws_slots = need ? static_cast<int32_t*>(workspace) : nullptr;
-  a.ws_counts = need ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + p.ws_slot_bytes)
-                     : nullptr;
+  a.ws_counts = need ? static_cast<unsigned*>(workspace) : nullptr;
+  a.ws_slots = need ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
+                    : nullptr;
   const CUtensorMap& ma = p.swap ? mw : mx;
   const CUtensorMap& mb = p.swap ? mx : mw;
   if (w4) {
