@@ -201,6 +201,28 @@ convrot_status convrot_w4a8_linear(const int8_t* Xq, const float* s_tok, const u
                                    convrot_stream_t stream);
 
 /*
+ * Allocation-free W8A8 linear.  The model cards have no counterpart: this is
+ * an interface addition for callers that cannot allocate device memory where
+ * they run the layer (plugins without an allocator, runtimes whose device
+ * memory is fixed after start-up, paths where an allocation would stall the
+ * device).  It computes exactly what convrot_int8_linear computes, with the
+ * same kernels, but takes the split-tile workspace from a fixed 24 MiB array
+ * inside the library instead of from the caller; it calls no allocator.
+ *  - Every GPU that loads the library holds that array until the process exits.
+ *  - The first call on a device looks up the array's device address
+ *    (set-up, once per device); make that first call before any stream capture.
+ *  - Shapes whose workspace exceeds 24 MiB are rejected with
+ *    CONVROT_ERR_WORKSPACE (on a 148-SM B200 every M <= 128 fits; larger M
+ *    with tiles split across CTAs does not - use convrot_int8_linear).
+ *  - All calls on a device share the array: each call clears the part that
+ *    must start at zero, and calls that overlap on the GPU race.
+ * Arguments, layouts and return codes otherwise as convrot_int8_linear.
+ */
+convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
+                                           const float* s_row, int M, int N, int K, void* Y,
+                                           convrot_stream_t stream);
+
+/*
  * Raw int32 accumulators of the same tensor-core kernels and work schedule
  * (including stream-K partial tiles), for exactness checks:
  * acc[m,n] = sum_k Xq[m,k] * Wq[n,k]   (int32 [M, N] out, 16-byte aligned).

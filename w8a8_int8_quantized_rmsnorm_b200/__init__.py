@@ -19,7 +19,7 @@ __all__ = [
     "ConvRotError", "lib", "convrot_version", "convrot_device_status",
     "convrot_quantize_weight", "convrot_quantize_weight_w4", "convrot_smoothquant_calibrate",
     "convrot_rotate_quant_act", "convrot_linear_workspace_bytes", "convrot_int8_linear",
-    "convrot_w4a8_linear", "convrot_int8_gemm_s32", "convrot_w4a8_gemm_s32",
+    "convrot_w4a8_linear", "convrot_int8_linear_noalloc", "convrot_int8_gemm_s32", "convrot_w4a8_gemm_s32",
     "Workspace", "ConvRotLinear",
 ]
 
@@ -191,6 +191,20 @@ def convrot_int8_linear(Xq, s_tok, Wq, s_row, out=None, workspace: Optional[Work
     _check("convrot_int8_linear", lib().convrot_int8_linear(
         _ptr(Xq), _ptr(s_tok), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), ws, wn,
         _stream(Xq.device)))
+    return Y
+
+
+def convrot_int8_linear_noalloc(Xq, s_tok, Wq, s_row, out=None):
+    """convrot_int8_linear without a caller workspace: the library's fixed
+    24 MiB per-device array serves as the split-tile workspace (for callers
+    that cannot allocate device memory where they run the layer).  Calls that
+    overlap on the GPU race on that array."""
+    M, N, K = _gemm_check(Xq, Wq, False)
+    _need(s_tok, torch.float32, "s_tok", 1)
+    _need(s_row, torch.float32, "s_row", 1)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    _check("convrot_int8_linear_noalloc", lib().convrot_int8_linear_noalloc(
+        _ptr(Xq), _ptr(s_tok), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), _stream(Xq.device)))
     return Y
 
 

@@ -48,6 +48,8 @@ SIGNATURES = {
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "convrot_w4a8_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
+    "convrot_int8_linear_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                            c_int, c_void_p, c_void_p]),
     "convrot_int8_gemm_s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
                                       c_void_p, c_size_t, c_void_p]),
     "convrot_w4a8_gemm_s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,

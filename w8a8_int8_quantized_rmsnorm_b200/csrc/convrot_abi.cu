@@ -508,3 +508,70 @@ convrot_status convrot_w4a8_gemm_s32(const int8_t* Xq, const uint8_t* Wq4, int M
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free variant of convrot_int8_linear.
+//
+// Some callers cannot allocate device memory at the point where they run a
+// linear layer: plugins that do not own an allocator, runtimes whose device
+// memory is planned once at start-up and must not grow afterwards, or code
+// paths where an allocation would synchronise the device.  For them this entry
+// point takes the GEMM's split-tile workspace from a fixed array that lives in
+// the library itself instead of from the caller.
+//
+// The array is a file-scope __device__ array of kStaticWorkspaceBytes; every
+// GPU that loads this library holds it until the process exits.  In host code
+// the array's name is only a host-side stand-in, never a device address, so
+// the device address is looked up with cudaGetSymbolAddress once per device
+// (the first call on a device does that set-up; make that first call before
+// any stream capture).  All calls on a device share the array and it keeps the
+// last call's contents: each call clears the tile counters that must start at
+// zero, and calls that overlap on the GPU (other streams, other threads) race
+// on it.
+// ===========================================================================
+constexpr size_t kStaticWorkspaceBytes = static_cast<size_t>(24) << 20;  // 24 MiB per device
+static __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
+
+namespace {
+std::mutex g_static_ws_mu;
+void* g_static_ws_ptr[64] = {nullptr};
+
+// Device address of g_static_workspace on `device` (the current device).
+convrot_status static_workspace_address(int device, void** out) {
+  std::lock_guard<std::mutex> g(g_static_ws_mu);
+  if (g_static_ws_ptr[device] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
+      return CONVROT_ERR_CUDA;
+    g_static_ws_ptr[device] = p;
+  }
+  *out = g_static_ws_ptr[device];
+  return CONVROT_OK;
+}
+}  // namespace
+
+extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const float* s_tok,
+                                                      const int8_t* Wq, const float* s_row,
+                                                      int M, int N, int K, void* Y,
+                                                      convrot_stream_t stream) {
+  const convrot_status sh = check_gemm_shape(M, N, K, false);
+  if (sh != CONVROT_OK) return sh;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  if (!Xq || !s_tok || !Wq || !s_row || !Y) return CONVROT_ERR_NULL;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(s_tok, 4) ||
+      !aligned(s_row, 4))
+    return CONVROT_ERR_ALIGN;
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
+  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms));
+  if (need > kStaticWorkspaceBytes) return CONVROT_ERR_WORKSPACE;  // shape too large for the array
+  void* ws = nullptr;
+  if (need > 0) {
+    const convrot_status a = static_workspace_address(d.device, &ws);
+    if (a != CONVROT_OK) return a;
+    if (cudaMemsetAsync(ws, 0, kCounterBytes, as_cuda(stream)) != cudaSuccess)
+      return CONVROT_ERR_CUDA;
+  }
+  return run_gemm(Xq, Wq, false, s_tok, s_row, M, N, K, Y, false, ws,
+                  need > 0 ? kStaticWorkspaceBytes : 0, as_cuda(stream));
+}
