@@ -7,12 +7,14 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/convrot.h"
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 #include "rowquant.cuh"
 
 using namespace convrot;
@@ -30,20 +32,18 @@ struct DeviceInfo {
 };
 
 DeviceInfo current_device() {
-  static std::mutex mu;
-  static int cached_sms[64] = {0};
+  static std::atomic<int> cached_sms[64];
   DeviceInfo d;
   if (cudaGetDevice(&d.device) != cudaSuccess || d.device < 0 || d.device >= 64) {
     d.device = -1;
     return d;
   }
-  std::lock_guard<std::mutex> g(mu);
-  if (cached_sms[d.device] == 0) {
-    int v = 0;
+  int v = cached_sms[d.device].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d.device) != cudaSuccess) v = 0;
-    cached_sms[d.device] = v;
+    cached_sms[d.device].store(v, std::memory_order_relaxed);
   }
-  d.sms = cached_sms[d.device];
+  d.sms = v;
   return d;
 }
 
@@ -66,22 +66,63 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D uint8 tensor [rows, row_bytes] (row stride = row_bytes), box
-// [box_rows, box_bytes], with or without the 128-byte swizzle.
-bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes,
-                 uint32_t box_rows, uint32_t box_bytes, bool swizzle128) {
+// A 2-D row-major tensor [rows, cols] of elements of `esize` bytes, box
+// [box_rows, box_cols], with or without the 128-byte swizzle.  Encoded maps
+// are kept in a small per-thread cache keyed by everything they encode, so a
+// steady stream of calls on the same buffers encodes nothing.
+struct MapKey {
+  const void* base;
+  uint64_t rows, cols;
+  uint32_t box_rows, box_cols;
+  int dtype, esize, swizzle;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && box_rows == o.box_rows &&
+           box_cols == o.box_cols && dtype == o.dtype && esize == o.esize && swizzle == o.swizzle;
+  }
+};
+
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, int esize,
+              CUtensorMapDataType dtype, uint32_t box_rows, uint32_t box_cols, bool swizzle128) {
+  constexpr int kCache = 32;
+  struct Entry {
+    MapKey key;
+    CUtensorMap map;
+    bool valid;
+  };
+  thread_local Entry cache[kCache] = {};
+  thread_local int next = 0;
+  const MapKey key{base, rows, cols, box_rows, box_cols, static_cast<int>(dtype), esize,
+                   swizzle128 ? 1 : 0};
+  for (int i = 0; i < kCache; ++i) {
+    if (cache[i].valid && cache[i].key == key) {
+      *map = cache[i].map;
+      return true;
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {row_bytes, rows};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r =
-      fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+      fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE,
          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (r != CUDA_SUCCESS) return false;
+  Entry& e = cache[next];
+  next = (next + 1) % kCache;
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
+  return true;
+}
+
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row_bytes,
+                 uint32_t box_rows, uint32_t box_bytes, bool swizzle128) {
+  return make_map(map, base, rows, row_bytes, 1, CU_TENSOR_MAP_DATA_TYPE_UINT8, box_rows,
+                  box_bytes, swizzle128);
 }
 
 convrot_status launch_status() {
@@ -119,9 +160,15 @@ template <bool ROT, int PRE, int QK, bool RES>
 convrot_status launch_rowquant_t(const RowQuantArgs& a, int threads, cudaStream_t st) {
   auto k = rowquant_kernel<ROT, PRE, QK, RES>;
   const DeviceInfo d = current_device();
-  int per_sm = 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, 0) != cudaSuccess)
-    return CONVROT_ERR_CUDA;
+  // occupancy per (device, block size in warps), computed once
+  static std::atomic<int> occ[64][33];
+  const int slot = std::min(32, (threads + 31) / 32);
+  int per_sm = d.device >= 0 ? occ[d.device][slot].load(std::memory_order_relaxed) : 0;
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, 0) != cudaSuccess)
+      return CONVROT_ERR_CUDA;
+    if (d.device >= 0) occ[d.device][slot].store(per_sm, std::memory_order_relaxed);
+  }
   const int row_blocks = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
   const int grid = std::max(1, std::min(row_blocks, std::max(1, per_sm) * std::max(1, d.sms)));
   k<<<grid, threads, 0, st>>>(a);
@@ -156,6 +203,7 @@ constexpr size_t kCounterBytes = 4096;
 
 struct GemmPlan {
   bool swap;
+  bool pair;  // CTA-pair kernel (256-row tiles); grid/units below count pairs
   int bn;
   int tilesA, tilesB, num_tiles, num_kb;
   int grid;
@@ -170,20 +218,26 @@ int pick_bn_swap(int M) {
   return 128;
 }
 
-GemmPlan plan_gemm(int M, int N, int K, int sms) {
+// `units` is the number of co-resident work units: SMs for the single-CTA
+// kernel, CTA pairs (clusters of two) for the pair kernel.
+GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs) {
   GemmPlan p{};
   p.swap = M <= 128;
+  p.pair = M > 256 && pairs > 0;
   p.bn = p.swap ? pick_bn_swap(M) : 256;
   const int rowsA = p.swap ? N : M;
   const int rowsB = p.swap ? M : N;
-  p.tilesA = (rowsA + GEMM_BM - 1) / GEMM_BM;
+  const int tileA = p.pair ? 256 : GEMM_BM;
+  p.tilesA = (rowsA + tileA - 1) / tileA;
   p.tilesB = (rowsB + p.bn - 1) / p.bn;
   p.num_tiles = p.tilesA * p.tilesB;
   p.num_kb = (K + GEMM_BK - 1) / GEMM_BK;
   const long long total = static_cast<long long>(p.num_tiles) * p.num_kb;
-  // at most 2 * grid tiles are split, so the fixed counter region always fits
-  const int max_grid = static_cast<int>(kCounterBytes / 4 / 2);
-  p.grid = static_cast<int>(std::min<long long>(std::min(std::max(1, sms), max_grid), total));
+  const int units = p.pair ? pairs : sms;
+  // at most 2 * units tiles are split (each with one counter per CTA of the
+  // unit), so the fixed counter region always fits
+  const int max_grid = static_cast<int>(kCounterBytes / 4 / 4);
+  p.grid = static_cast<int>(std::min<long long>(std::min(std::max(1, units), max_grid), total));
   const int waves = p.num_tiles / p.grid;
   p.dp_tiles = waves >= 2 ? (waves - 1) * p.grid : 0;
   const int sk_tiles = p.num_tiles - p.dp_tiles;
@@ -192,9 +246,75 @@ GemmPlan plan_gemm(int M, int N, int K, int sms) {
   p.sk_r = p.sk_iters % p.grid;
   // a stream-K region whose iterations split evenly into whole tiles needs no workspace
   const bool whole = p.sk_r == 0 && p.sk_q % p.num_kb == 0;
-  p.ws_slot_bytes = whole ? 0 : static_cast<size_t>(2) * p.grid * GEMM_BM * p.bn * 4;
-  p.ws_count_bytes = whole ? 0 : static_cast<size_t>(sk_tiles) * 4;
+  const int ctas_per_unit = p.pair ? 2 : 1;
+  p.ws_slot_bytes =
+      whole ? 0 : static_cast<size_t>(2) * p.grid * ctas_per_unit * GEMM_BM * p.bn * 4;
+  p.ws_count_bytes = whole ? 0 : static_cast<size_t>(sk_tiles) * ctas_per_unit * 4;
   return p;
+}
+
+// Co-resident clusters of two CTAs of the pair kernel (once per device).
+template <bool W4, int EPI>
+int pair_units(int device) {
+  static std::atomic<int> cached[64];
+  if (device < 0 || device >= 64) return 0;
+  int v = cached[device].load(std::memory_order_relaxed);
+  if (v != 0) return v;
+  using SM = Gemm2Smem<W4>;
+  auto k = gemm2sm_kernel<W4, EPI>;
+  const int avail = 227 * 1024 - 1024 - SM::total(0);
+  const int stages = std::max(2, std::min(GEMM_MAX_STAGES, avail / SM::STAGE));
+  const int smem = SM::total(stages) + 1024;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(W4 ? 448 : 320, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, k, &cfg) != cudaSuccess || clusters <= 0) {
+    cudaGetLastError();
+    clusters = -1;  // pair kernel unavailable: fall back to single-CTA tiles
+  }
+  cached[device].store(clusters, std::memory_order_relaxed);
+  return clusters;
+}
+
+int pair_units_for(bool w4, bool s32, int device) {
+  if (w4) return s32 ? pair_units<true, EPI_S32>(device) : pair_units<true, EPI_BF16>(device);
+  return s32 ? pair_units<false, EPI_S32>(device) : pair_units<false, EPI_BF16>(device);
+}
+
+template <bool W4, int EPI>
+convrot_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
+                                GemmArgs a, int pairs, cudaStream_t st) {
+  using SM = Gemm2Smem<W4>;
+  auto k = gemm2sm_kernel<W4, EPI>;
+  const int avail = 227 * 1024 - 1024 - SM::total(0);
+  const int stages = std::max(2, std::min(GEMM_MAX_STAGES, avail / SM::STAGE));
+  a.stages = stages;
+  const int smem = SM::total(stages) + 1024;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(W4 ? 448 : 320, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k, ma, mb, my, a) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return launch_status();
 }
 
 // Workspace layout: a fixed region of tile counters at offset 0 (left at zero
@@ -207,13 +327,14 @@ size_t ws_bytes(const GemmPlan& p) {
 }
 
 template <int BN, bool SWAP, bool W4, int EPI>
-convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs a, int grid,
-                             cudaStream_t st) {
+convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
+                             GemmArgs a, int grid, cudaStream_t st) {
   using SM = GemmSmem<BN, W4, SWAP>;
   auto k = gemm_kernel<BN, SWAP, W4, EPI>;
-  // at least ~116 KB so that a second CTA never shares the SM's TMEM
-  const int budget = 200 * 1024;
-  int stages = std::min(GEMM_MAX_STAGES, budget / SM::STAGE);
+  // as many stages as fit next to the epilogue staging and the barriers in
+  // 227 KB; at least ~116 KB so that a second CTA never shares the SM's TMEM
+  const int avail = 227 * 1024 - 1024 - SM::total(0);
+  int stages = std::min(GEMM_MAX_STAGES, avail / SM::STAGE);
   stages = std::max(2, stages);
   a.stages = stages;
   const int smem = std::max(SM::total(stages) + 1024, 116 * 1024);
@@ -226,19 +347,20 @@ convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, GemmA
     configured_device_mask |= bit;
   }
   constexpr int threads = W4 ? 320 : 192;
-  k<<<grid, threads, smem, st>>>(ma, mb, a);
+  k<<<grid, threads, smem, st>>>(ma, mb, my, a);
   return launch_status();
 }
 
 template <bool SWAP, bool W4, int EPI>
 convrot_status launch_gemm_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mb,
-                              const GemmArgs& a, int grid, cudaStream_t st) {
-  if (!SWAP) return launch_gemm_t<256, false, W4, EPI>(ma, mb, a, grid, st);
+                              const CUtensorMap& my, const GemmArgs& a, int grid,
+                              cudaStream_t st) {
+  if (!SWAP) return launch_gemm_t<256, false, W4, EPI>(ma, mb, my, a, grid, st);
   switch (bn) {
-    case 16: return launch_gemm_t<16, true, W4, EPI>(ma, mb, a, grid, st);
-    case 32: return launch_gemm_t<32, true, W4, EPI>(ma, mb, a, grid, st);
-    case 64: return launch_gemm_t<64, true, W4, EPI>(ma, mb, a, grid, st);
-    default: return launch_gemm_t<128, true, W4, EPI>(ma, mb, a, grid, st);
+    case 16: return launch_gemm_t<16, true, W4, EPI>(ma, mb, my, a, grid, st);
+    case 32: return launch_gemm_t<32, true, W4, EPI>(ma, mb, my, a, grid, st);
+    case 64: return launch_gemm_t<64, true, W4, EPI>(ma, mb, my, a, grid, st);
+    default: return launch_gemm_t<128, true, W4, EPI>(ma, mb, my, a, grid, st);
   }
 }
 
@@ -247,21 +369,31 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const GemmPlan p = plan_gemm(M, N, K, d.sms);
+  const GemmPlan p = plan_gemm(M, N, K, d.sms, pair_units_for(w4, s32_out, d.device));
   const size_t need = ws_bytes(p);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CONVROT_ERR_WORKSPACE;
   if (need > 0 && !aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
 
   const int bn = p.bn;
   CUtensorMap mx, mw;
-  // activations: int8 [M, K]; weights: int8 [N, K] or packed [N, K/2]
+  // activations: int8 [M, K]; weights: int8 [N, K] or packed [N, K/2].  Each
+  // CTA of a pair loads 128 rows of each operand.
   const uint32_t x_box_rows = p.swap ? bn : GEMM_BM;
-  const uint32_t w_box_rows = p.swap ? GEMM_BM : bn;
+  const uint32_t w_box_rows = (p.swap || p.pair) ? GEMM_BM : bn;
   if (!make_map_u8(&mx, Xq, M, K, x_box_rows, GEMM_BK, true)) return CONVROT_ERR_CUDA;
   if (w4) {
     if (!make_map_u8(&mw, Wq, N, K / 2, w_box_rows, GEMM_BK / 2, false)) return CONVROT_ERR_CUDA;
   } else {
     if (!make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK, true)) return CONVROT_ERR_CUDA;
+  }
+
+  // output map for the non-swap epilogue's TMA stores: rows of 128 bytes
+  CUtensorMap my;
+  std::memset(&my, 0, sizeof(my));
+  if (!p.swap) {
+    const bool ok = s32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_INT32, 32, 32, true)
+                            : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, 64, true);
+    if (!ok) return CONVROT_ERR_CUDA;
   }
 
   GemmArgs a{};
@@ -280,24 +412,32 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
   a.sk_r = p.sk_r;
   a.s_tok = s_tok;
   a.s_row = s_row;
+  a.srow_vec = (s_row != nullptr && aligned(s_row, 16)) ? 1 : 0;
   a.out = out;
   a.ws_counts = need ? static_cast<unsigned*>(workspace) : nullptr;
   a.ws_slots = need ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
                     : nullptr;
   const CUtensorMap& ma = p.swap ? mw : mx;
   const CUtensorMap& mb = p.swap ? mx : mw;
+  if (p.pair) {
+    if (w4)
+      return s32_out ? launch_gemm_pair<true, EPI_S32>(ma, mb, my, a, p.grid, st)
+                     : launch_gemm_pair<true, EPI_BF16>(ma, mb, my, a, p.grid, st);
+    return s32_out ? launch_gemm_pair<false, EPI_S32>(ma, mb, my, a, p.grid, st)
+                   : launch_gemm_pair<false, EPI_BF16>(ma, mb, my, a, p.grid, st);
+  }
   if (w4) {
     if (s32_out)
-      return p.swap ? launch_gemm_bn<true, true, EPI_S32>(bn, ma, mb, a, p.grid, st)
-                    : launch_gemm_bn<false, true, EPI_S32>(bn, ma, mb, a, p.grid, st);
-    return p.swap ? launch_gemm_bn<true, true, EPI_BF16>(bn, ma, mb, a, p.grid, st)
-                  : launch_gemm_bn<false, true, EPI_BF16>(bn, ma, mb, a, p.grid, st);
+      return p.swap ? launch_gemm_bn<true, true, EPI_S32>(bn, ma, mb, my, a, p.grid, st)
+                    : launch_gemm_bn<false, true, EPI_S32>(bn, ma, mb, my, a, p.grid, st);
+    return p.swap ? launch_gemm_bn<true, true, EPI_BF16>(bn, ma, mb, my, a, p.grid, st)
+                  : launch_gemm_bn<false, true, EPI_BF16>(bn, ma, mb, my, a, p.grid, st);
   }
   if (s32_out)
-    return p.swap ? launch_gemm_bn<true, false, EPI_S32>(bn, ma, mb, a, p.grid, st)
-                  : launch_gemm_bn<false, false, EPI_S32>(bn, ma, mb, a, p.grid, st);
-  return p.swap ? launch_gemm_bn<true, false, EPI_BF16>(bn, ma, mb, a, p.grid, st)
-                : launch_gemm_bn<false, false, EPI_BF16>(bn, ma, mb, a, p.grid, st);
+    return p.swap ? launch_gemm_bn<true, false, EPI_S32>(bn, ma, mb, my, a, p.grid, st)
+                  : launch_gemm_bn<false, false, EPI_S32>(bn, ma, mb, my, a, p.grid, st);
+  return p.swap ? launch_gemm_bn<true, false, EPI_BF16>(bn, ma, mb, my, a, p.grid, st)
+                : launch_gemm_bn<false, false, EPI_BF16>(bn, ma, mb, my, a, p.grid, st);
 }
 
 convrot_status check_gemm_shape(int M, int N, int K, bool w4) {
@@ -447,7 +587,8 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits) {
   if (M == 0 || N == 0) return 0;
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return 0;
-  return ws_bytes(plan_gemm(M, N, K, d.sms));
+  // the bf16 and int32 outputs share the schedule, so either plan gives the size
+  return ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(weight_bits == 4, false, d.device)));
 }
 
 static convrot_status linear_common(const int8_t* Xq, const float* s_tok, const void* Wq,
@@ -563,7 +704,7 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
     return CONVROT_ERR_ALIGN;
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms));
+  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(false, false, d.device)));
   if (need > kStaticWorkspaceBytes) return CONVROT_ERR_WORKSPACE;  // shape too large for the array
   void* ws = nullptr;
   if (need > 0) {

@@ -64,6 +64,7 @@ struct GemmArgs {
   int sk_q, sk_r;    // stream-K split: first sk_r CTAs get sk_q + 1 iterations
   const float* s_tok;
   const float* s_row;
+  int srow_vec;  // s_row is 16-byte aligned: vector loads in the epilogue
   void* out;
   int32_t* ws_slots;     // [2 * gridDim.x][BM * BN] partial tiles
   unsigned* ws_counts;   // [num_tiles - dp_tiles]
@@ -81,10 +82,11 @@ struct Schedule {
   int dp_next;
   int sk_begin, sk_end, sk_cur;
 
-  __device__ void init(const GemmArgs& a) {
+  // unit = CTA (or CTA pair) index, nunits = number of units in the grid
+  __device__ void init(const GemmArgs& a, int unit, int nunits) {
     p = &a;
-    cta = blockIdx.x;
-    ncta = gridDim.x;
+    cta = unit;
+    ncta = nunits;
     dp_next = cta;
     sk_begin = cta * a.sk_q + min(cta, a.sk_r);
     sk_end = sk_begin + a.sk_q + (cta < a.sk_r ? 1 : 0);
@@ -134,10 +136,6 @@ __device__ __forceinline__ void tile_coords(const GemmArgs& a, int tile, int& ta
   tb = local / ga;
 }
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -151,10 +149,13 @@ struct GemmSmem {
   static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
   static constexpr int P_BYTES = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 weight tile
   static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+  // non-swap epilogue: per epilogue warp two 4 KB staging buffers (32 rows x 128 B)
+  static constexpr int STAGING = SWAP ? 0 : 4 * 2 * 4096;
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;  // TMEM columns per accumulator buffer
   static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
   static constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
-  __host__ __device__ static int bar_offset(int stages) { return stages * STAGE; }
+  __host__ __device__ static int staging_offset(int stages) { return stages * STAGE; }
+  __host__ __device__ static int bar_offset(int stages) { return stages * STAGE + STAGING; }
   // full, empty, conv: stages each; tmem_full, tmem_empty: 2 each; + scalars
   __host__ __device__ static int total(int stages) {
     return bar_offset(stages) + (3 * GEMM_MAX_STAGES + 6) * 8 + 64;
@@ -164,7 +165,7 @@ struct GemmSmem {
 template <int BN, bool SWAP, bool W4, int EPI>
 __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                GemmArgs a) {
+                const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = GemmSmem<BN, W4, SWAP>;
   constexpr int CW = SM::CW;
   constexpr uint32_t IDESC = idesc_s8s8s32(GEMM_BM, BN);
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (!SWAP) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, SM::TMEM_COLS);
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   Schedule sched;
-  sched.init(a);
+  sched.init(a, blockIdx.x, gridDim.x);
   Segment seg;
 
   if (warp == 0) {
@@ -316,6 +318,10 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
       __syncwarp();
       return r;
     };
+    // output columns per staged 128-byte row (non-swap path)
+    constexpr int OC = (EPI == EPI_BF16) ? 64 : 32;
+    uint8_t* stage_buf = smem + SM::staging_offset(S) + q * 8192;
+    int sbuf = 0;
     while (sched.next(seg)) {
       const uint32_t b = local & 1u;
       const uint32_t use = local >> 1;
@@ -329,7 +335,8 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
       const int arow = ta * GEMM_BM + 32 * q + lane;  // operand-A row of this thread
 
       if (seg.partial) {
-        // write this CTA's partial tile to its slot
+        // write this CTA's partial tile to its slot: for each 32-column chunk c
+        // and warp q, 8 x 16 bytes per lane, consecutive lanes consecutive
         int32_t* slot = a.ws_slots + static_cast<size_t>(seg.slot) * (GEMM_BM * BN);
 #pragma unroll 1
         for (int c = 0; c < BN / CW; ++c) {
@@ -376,72 +383,139 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
           c_lo = sk_owner(a, u * a.num_kb);
           c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
         }
+        if (!SWAP) {
+          // ---- rows of the output tile: staged through shared memory, TMA stores
+          const int m = arow;
+          const int m0 = ta * GEMM_BM + 32 * q;
+          float st = 0.f;
+          if (EPI == EPI_BF16 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
 #pragma unroll 1
-        for (int c = 0; c < BN / CW; ++c) {
-          uint32_t r[32];
-          if (!seg.partial) {
-            if (CW == 32) {
-              tmem_ld_32x32b_x32(tbase + c * CW, r);
+          for (int oc = 0; oc < BN / OC; ++oc) {
+            uint32_t r0[32], r1[32];
+            if (!seg.partial) {
+              tmem_ld_32x32b_x32(tbase + oc * OC, r0);
+              if (OC == 64) tmem_ld_32x32b_x32(tbase + oc * OC + 32, r1);
+              tmem_ld_wait();
             } else {
-              tmem_ld_32x32b_x16(tbase + c * CW, r);
-            }
-            tmem_ld_wait();
-          } else {
 #pragma unroll
-            for (int j = 0; j < CW; ++j) r[j] = 0u;
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              const int slot_id = 2 * cc + (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
-              const uint4* src = reinterpret_cast<const uint4*>(
-                                     a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN)) +
-                                 (c * 4 + q) * (CW / 4) * 32 + lane;
-#pragma unroll
-              for (int j4 = 0; j4 < CW / 4; ++j4) {
-                const uint4 v = __ldcg(src + j4 * 32);
-                r[4 * j4] += v.x;
-                r[4 * j4 + 1] += v.y;
-                r[4 * j4 + 2] += v.z;
-                r[4 * j4 + 3] += v.w;
+              for (int j = 0; j < 32; ++j) {
+                r0[j] = 0u;
+                r1[j] = 0u;
               }
-            }
-          }
-          // ---- store one CW-column chunk
-          if (!SWAP) {
-            const int m = arow;
-            const int n0 = tb * BN + c * CW;
-            if (m < a.M) {
-              if (EPI == EPI_BF16) {
-                const float st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
-                __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(m) * a.N;
+              for (int cc = c_lo; cc <= c_hi; ++cc) {
+                const int slot_id = 2 * cc + (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
+                const uint4* base = reinterpret_cast<const uint4*>(
+                    a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN));
+                const int c0 = oc * (OC / 32);
+                uint4 v0[8], v1[8];
 #pragma unroll
-                for (int j8 = 0; j8 < CW / 8; ++j8) {
-                  const int n = n0 + 8 * j8;
-                  if (n < a.N) {
-                    uint32_t w[4];
+                for (int j4 = 0; j4 < 8; ++j4) {
+                  v0[j4] = __ldcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane);
+                  if (OC == 64) v1[j4] = __ldcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane);
+                }
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                      const float y0 = static_cast<float>(static_cast<int32_t>(r[8 * j8 + 2 * h])) * st * __ldg(a.s_row + n + 2 * h);
-                      const float y1 = static_cast<float>(static_cast<int32_t>(r[8 * j8 + 2 * h + 1])) * st * __ldg(a.s_row + n + 2 * h + 1);
-                      w[h] = pack_bf16x2(y0, y1);
-                    }
-                    *reinterpret_cast<uint4*>(y + n) = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int j4 = 0; j4 < 8; ++j4) {
+                  r0[4 * j4] += v0[j4].x;
+                  r0[4 * j4 + 1] += v0[j4].y;
+                  r0[4 * j4 + 2] += v0[j4].z;
+                  r0[4 * j4 + 3] += v0[j4].w;
+                  if (OC == 64) {
+                    r1[4 * j4] += v1[j4].x;
+                    r1[4 * j4 + 1] += v1[j4].y;
+                    r1[4 * j4 + 2] += v1[j4].z;
+                    r1[4 * j4 + 3] += v1[j4].w;
                   }
                 }
+              }
+            }
+            uint8_t* buf = stage_buf + sbuf * 4096;
+            if (lane == 0) bulk_wait_group_read<1>();  // the store from two chunks ago has read buf
+            __syncwarp();
+            const int sw = lane & 7;
+            if (EPI == EPI_BF16) {
+              const int n0 = tb * BN + oc * OC;
+#pragma unroll
+              for (int c16 = 0; c16 < 8; ++c16) {
+                const uint32_t* rr = c16 < 4 ? r0 : r1;
+                const int jb = (c16 & 3) * 8;
+                const int n = n0 + c16 * 8;
+                float sr[8];
+                if (n < a.N) {
+                  if (a.srow_vec) {
+                    const float4 s0 = __ldg(reinterpret_cast<const float4*>(a.s_row + n));
+                    const float4 s1 = __ldg(reinterpret_cast<const float4*>(a.s_row + n + 4));
+                    sr[0] = s0.x; sr[1] = s0.y; sr[2] = s0.z; sr[3] = s0.w;
+                    sr[4] = s1.x; sr[5] = s1.y; sr[6] = s1.z; sr[7] = s1.w;
+                  } else {
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) sr[h] = __ldg(a.s_row + n + h);
+                  }
+                } else {
+#pragma unroll
+                  for (int h = 0; h < 8; ++h) sr[h] = 0.f;
+                }
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const float y0 = static_cast<float>(static_cast<int32_t>(rr[jb + 2 * h])) * st * sr[2 * h];
+                  const float y1 = static_cast<float>(static_cast<int32_t>(rr[jb + 2 * h + 1])) * st * sr[2 * h + 1];
+                  w[h] = pack_bf16x2(y0, y1);
+                }
+                st_shared_v4(buf + lane * 128 + ((c16 ^ sw) << 4), w[0], w[1], w[2], w[3]);
+              }
+            } else {
+              const int sh = W4 ? 4 : 0;
+#pragma unroll
+              for (int c16 = 0; c16 < 8; ++c16) {
+                st_shared_v4(buf + lane * 128 + ((c16 ^ sw) << 4),
+                             static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16]) >> sh),
+                             static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16 + 1]) >> sh),
+                             static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16 + 2]) >> sh),
+                             static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16 + 3]) >> sh));
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, buf, tb * BN + oc * OC, m0);
+              bulk_commit_group();
+            }
+            sbuf ^= 1;
+          }
+        } else {
+          // ---- swapped roles: lanes are weight rows n, columns are tokens m;
+          // for each token the warp writes 32 consecutive outputs (64 bytes)
+          const int n = arow;
+#pragma unroll 1
+          for (int c = 0; c < BN / CW; ++c) {
+            uint32_t r[32];
+            if (!seg.partial) {
+              if (CW == 32) {
+                tmem_ld_32x32b_x32(tbase + c * CW, r);
               } else {
-                int32_t* y = reinterpret_cast<int32_t*>(a.out) + static_cast<size_t>(m) * a.N;
+                tmem_ld_32x32b_x16(tbase + c * CW, r);
+              }
+              tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int j = 0; j < CW; ++j) r[j] = 0u;
+              for (int cc = c_lo; cc <= c_hi; ++cc) {
+                const int slot_id = 2 * cc + (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
+                const uint4* src = reinterpret_cast<const uint4*>(
+                                       a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN)) +
+                                   (c * 4 + q) * (CW / 4) * 32 + lane;
+                uint4 v[CW / 4];
+#pragma unroll
+                for (int j4 = 0; j4 < CW / 4; ++j4) v[j4] = __ldcg(src + j4 * 32);
 #pragma unroll
                 for (int j4 = 0; j4 < CW / 4; ++j4) {
-                  const int n = n0 + 4 * j4;
-                  if (n < a.N) {
-                    const int sh = W4 ? 4 : 0;
-                    *reinterpret_cast<int4*>(y + n) =
-                        make_int4(static_cast<int32_t>(r[4 * j4]) >> sh, static_cast<int32_t>(r[4 * j4 + 1]) >> sh,
-                                  static_cast<int32_t>(r[4 * j4 + 2]) >> sh, static_cast<int32_t>(r[4 * j4 + 3]) >> sh);
-                  }
+                  r[4 * j4] += v[j4].x;
+                  r[4 * j4 + 1] += v[j4].y;
+                  r[4 * j4 + 2] += v[j4].z;
+                  r[4 * j4 + 3] += v[j4].w;
                 }
               }
             }
-          } else {
-            const int n = arow;  // weight row
             const int m0 = tb * BN + c * CW;
             if (n < a.N) {
               if (EPI == EPI_BF16) {
@@ -474,6 +548,8 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
       }
       ++local;
     }
+    // every output store must be complete before the CTA exits
+    if (!SWAP && lane == 0) bulk_wait_group<0>();
   } else if (W4) {
     // ------------------------------------------------------------ int4 unpack
     const int ct = threadIdx.x - 192;  // 0..127

@@ -1,0 +1,424 @@
+// W8A8 / W4A8 ConvRot linear on CTA pairs (tcgen05 cta_group::2), for M > 256.
+//
+// Same arithmetic as gemm_kernel ("MOSS-Image Qwen3.5-9B text encoder, INT8
+// (W8A8, ConvRot)", file table, "Matmul" row; int4 layout of "MossInt4",
+// "Format"):
+//   acc[m, n] = sum_k Xq[m, k] * Wq[n, k];  Y[m, n] = bf16(float(acc) * s_tok[m] * s_row[n])
+//
+// Two CTAs of a cluster share one 256 x 256 output tile.  Each CTA stages its
+// own 128 rows of activations (A) and its own 128 rows of weights (B, half of
+// the tile's N) - 32 KB per 128-byte K step instead of the 48 KB one CTA needs
+// for a 128 x 256 tile - so six stages fit and each SM pulls 64 B/clk at the
+// tensor pipe's rate.  One thread of the leader CTA issues
+// tcgen05.mma.cta_group::2 (256 x 256 x 32 int8): the hardware reads A and B
+// from both CTAs' shared memory and writes each CTA's 128 accumulator rows x
+// 256 columns into that CTA's TMEM.  TMA loads never use cluster multicast:
+// each CTA loads its own tiles.
+//
+// Roles per CTA:
+//   warp 0       TMA producer (int8: completion counted on the leader's barrier)
+//   warp 1       TMEM allocation (pair-wide); in the leader, the MMA issuer
+//   warps 2-9    epilogue: two warps per TMEM lane quadrant, each 128 columns;
+//                bf16 (or int32) rows staged in shared memory, TMA stores
+//   warps 10-13  (int4 only) unpack nibbles of this CTA's weight rows
+// Work split, stream-K partial tiles and their workspace protocol are those of
+// gemm_kernel with a CTA pair as the unit; each CTA of the pair fixes up its
+// own 128 rows of a split tile.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace convrot {
+
+constexpr int PAIR_EPI_WARPS = 8;
+
+template <bool W4>
+struct Gemm2Smem {
+  static constexpr int A_BYTES = 128 * GEMM_BK;
+  static constexpr int B_BYTES = 128 * GEMM_BK;
+  static constexpr int P_BYTES = W4 ? 128 * (GEMM_BK / 2) : 0;
+  static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int STAGING = PAIR_EPI_WARPS * 4096;
+  static constexpr int TMEM_COLS = 512;
+  __host__ __device__ static int staging_offset(int stages) { return stages * STAGE; }
+  __host__ __device__ static int bar_offset(int stages) { return stages * STAGE + STAGING; }
+  __host__ __device__ static int total(int stages) {
+    return bar_offset(stages) + (3 * GEMM_MAX_STAGES + 8) * 8 + 64;
+  }
+};
+
+template <bool W4, int EPI>
+__global__ void __launch_bounds__(W4 ? 448 : 320, 1)
+    gemm2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
+  using SM = Gemm2Smem<W4>;
+  constexpr int BN = 256;
+  constexpr uint32_t IDESC = idesc_s8s8s32(256, BN);
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int S = a.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::bar_offset(S));
+  uint64_t* empty = full + GEMM_MAX_STAGES;
+  uint64_t* conv = empty + GEMM_MAX_STAGES;
+  uint64_t* tmem_full = conv + GEMM_MAX_STAGES;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* drain = tmem_empty + 2;
+  uint64_t* epi_sync = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&conv[s], 8);  // 4 converter warps in each CTA (leader's barrier)
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tmem_full[b], 1);
+      mbar_init(&tmem_empty[b], 2 * PAIR_EPI_WARPS);  // both CTAs' epilogue warps (leader's)
+    }
+    mbar_init(drain, 1);
+    mbar_init(epi_sync, PAIR_EPI_WARPS);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, SM::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  Schedule sched;
+  sched.init(a, pair, npairs);
+  Segment seg;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_b = policy_evict_first();
+      uint32_t it = 0;
+      bool ok = true;
+      while (ok && sched.next(seg)) {
+        int ta, tb;
+        tile_coords(a, seg.tile, ta, tb);
+        const int arow = ta * 256 + static_cast<int>(rank) * 128;
+        const int brow = tb * BN + static_cast<int>(rank) * 128;
+        for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, SITE_PROD_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * SM::STAGE;
+          if (W4) {
+            // each CTA converts its own weight rows: completion on its own barrier
+            mbar_arrive_expect_tx(&full[s], SM::A_BYTES + SM::P_BYTES);
+            tma_load_2d(st, &tmA, &full[s], kb * GEMM_BK, arow, pol_a);
+            tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], kb * (GEMM_BK / 2), brow,
+                        pol_b);
+          } else {
+            // both CTAs' tiles complete on the leader's barrier, which the leader arms
+            const uint32_t lead_full = mapa_shared(smem_addr(&full[s]), 0);
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (SM::A_BYTES + SM::B_BYTES));
+            tma_load_2d_pair(st, &tmA, lead_full, kb * GEMM_BK, arow, pol_a);
+            tma_load_2d_pair(st + SM::A_BYTES, &tmB, lead_full, kb * GEMM_BK, brow, pol_b);
+          }
+        }
+      }
+      if (W4) {
+        // drain: no copy may still be landing in shared memory when the CTA exits
+        const uint32_t n_issued = it;
+        const uint32_t first = n_issued > static_cast<uint32_t>(S) ? n_issued - S : 0u;
+        for (uint32_t j = first; j < n_issued; ++j) {
+          int dummy = 0;
+          mbar_wait(&full[j % S], (j / S) & 1u, &dummy, SITE_DRAIN);
+        }
+      }
+      // int8: the leader's MMA thread consumed every stage, so both CTAs' copies
+      // have landed before it passes the final pair barrier
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && rank == 0) {
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      while (ok && sched.next(seg)) {
+        const uint32_t b = local & 1u;
+        const uint32_t use = local >> 1;
+        if (!mbar_wait(&tmem_empty[b], (use & 1u) ^ 1u, abort_flag, SITE_MMA_TMEM)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + b * BN;
+        for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1u;
+          if (!mbar_wait(W4 ? &conv[s] : &full[s], ph, abort_flag, SITE_MMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(smem + s * SM::STAGE);
+          const uint32_t sb = sa + SM::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
+            mma_s8_pair(d, sw128_kmajor_desc(sa + k * GEMM_UMMA_K),
+                        sw128_kmajor_desc(sb + k * GEMM_UMMA_K), IDESC,
+                        (kb > seg.kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair_mc(&empty[s], 0x3);
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&tmem_full[b], 0x3);
+        ++local;
+      }
+      // every MMA this thread issued must be complete before TMEM is released
+      mma_commit_pair(drain);
+      int never = 0;
+      mbar_wait(drain, 0u, &never, SITE_DRAIN);
+    }
+  } else if (warp < 2 + PAIR_EPI_WARPS) {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;          // 0..7
+    const int q = warp & 3;           // TMEM lane quadrant this warp may access
+    const int h = ew >> 2;            // column half of the tile: 128 columns each
+    uint32_t local = 0;
+    uint32_t sync_phase = 0;
+    auto epi_rendezvous = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(epi_sync);
+      const bool r = mbar_wait(epi_sync, sync_phase & 1u, abort_flag, SITE_EPI_SYNC);
+      ++sync_phase;
+      __syncwarp();
+      return r;
+    };
+    constexpr int OC = (EPI == EPI_BF16) ? 64 : 32;  // output columns per 128-byte staged row
+    uint8_t* buf = smem + SM::staging_offset(S) + ew * 4096;
+    while (sched.next(seg)) {
+      const uint32_t b = local & 1u;
+      const uint32_t use = local >> 1;
+      const bool got = mbar_wait(&tmem_full[b], use & 1u, abort_flag, SITE_EPI_FULL);
+      __syncwarp();
+      if (!got) break;
+      tc_fence_after();
+      int ta, tb;
+      tile_coords(a, seg.tile, ta, tb);
+      const int m0 = ta * 256 + static_cast<int>(rank) * 128 + 32 * q;  // first row of this warp
+      const int ncol0 = tb * BN + h * 128;                              // first column of this warp
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * BN + h * 128;
+      const uint32_t lead_tmem_empty = mapa_shared(smem_addr(&tmem_empty[b]), 0);
+
+      if (seg.partial) {
+        int32_t* slot = a.ws_slots + static_cast<size_t>(2 * (2 * sched.cta + rank) + (seg.slot & 1)) *
+                                         (GEMM_BM * BN);
+#pragma unroll 1
+        for (int cl = 0; cl < 4; ++cl) {  // this warp's 32-column chunks
+          const int c = h * 4 + cl;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + cl * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            uint4* dst = reinterpret_cast<uint4*>(slot) + ((c * 4 + q) * 8 + j4) * 32 + lane;
+            *dst = make_uint4(r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+          }
+        }
+      }
+      bool finalize = !seg.partial;
+      if (seg.partial) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);
+        __threadfence();
+        if (!epi_rendezvous()) break;
+        if (ew == 0 && lane == 0) {
+          const int u = seg.tile - a.dp_tiles;
+          const int c_lo = sk_owner(a, u * a.num_kb);
+          const int c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
+          const unsigned prev = atomicAdd(&a.ws_counts[2 * u + rank], 1u);
+          const bool last = prev + 1u == static_cast<unsigned>(c_hi - c_lo + 1);
+          if (last) a.ws_counts[2 * u + rank] = 0u;
+          *last_flag = last ? 1 : 0;
+        }
+        if (!epi_rendezvous()) break;
+        finalize = *last_flag != 0;
+        if (finalize) __threadfence();
+      }
+      if (finalize) {
+        int c_lo = 0, c_hi = -1, u = 0;
+        if (seg.partial) {
+          u = seg.tile - a.dp_tiles;
+          c_lo = sk_owner(a, u * a.num_kb);
+          c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
+        }
+        const int m = m0 + lane;
+        float st = 0.f;
+        if (EPI == EPI_BF16 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
+#pragma unroll 1
+        for (int oc = 0; oc < 128 / OC; ++oc) {
+          uint32_t r0[32], r1[32];
+          if (!seg.partial) {
+            tmem_ld_32x32b_x32(tbase + oc * OC, r0);
+            if (OC == 64) tmem_ld_32x32b_x32(tbase + oc * OC + 32, r1);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              r0[j] = 0u;
+              r1[j] = 0u;
+            }
+            const int c0 = h * 4 + oc * (OC / 32);
+            for (int cc = c_lo; cc <= c_hi; ++cc) {
+              const int slot_id = 2 * (2 * cc + static_cast<int>(rank)) +
+                                  (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
+              const uint4* base = reinterpret_cast<const uint4*>(
+                  a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN));
+              uint4 v0[8], v1[8];
+#pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+                v0[j4] = __ldcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane);
+                if (OC == 64) v1[j4] = __ldcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane);
+              }
+#pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+                r0[4 * j4] += v0[j4].x;
+                r0[4 * j4 + 1] += v0[j4].y;
+                r0[4 * j4 + 2] += v0[j4].z;
+                r0[4 * j4 + 3] += v0[j4].w;
+                if (OC == 64) {
+                  r1[4 * j4] += v1[j4].x;
+                  r1[4 * j4 + 1] += v1[j4].y;
+                  r1[4 * j4 + 2] += v1[j4].z;
+                  r1[4 * j4 + 3] += v1[j4].w;
+                }
+              }
+            }
+          }
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read buf
+          __syncwarp();
+          const int sw = lane & 7;
+          if (EPI == EPI_BF16) {
+            const int n0 = ncol0 + oc * OC;
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) {
+              const uint32_t* rr = c16 < 4 ? r0 : r1;
+              const int jb = (c16 & 3) * 8;
+              const int n = n0 + c16 * 8;
+              float sr[8];
+              if (n < a.N) {
+                if (a.srow_vec) {
+                  const float4 s0 = __ldg(reinterpret_cast<const float4*>(a.s_row + n));
+                  const float4 s1 = __ldg(reinterpret_cast<const float4*>(a.s_row + n + 4));
+                  sr[0] = s0.x; sr[1] = s0.y; sr[2] = s0.z; sr[3] = s0.w;
+                  sr[4] = s1.x; sr[5] = s1.y; sr[6] = s1.z; sr[7] = s1.w;
+                } else {
+#pragma unroll
+                  for (int hh = 0; hh < 8; ++hh) sr[hh] = __ldg(a.s_row + n + hh);
+                }
+              } else {
+#pragma unroll
+                for (int hh = 0; hh < 8; ++hh) sr[hh] = 0.f;
+              }
+              uint32_t w[4];
+#pragma unroll
+              for (int hh = 0; hh < 4; ++hh) {
+                const float y0 = static_cast<float>(static_cast<int32_t>(rr[jb + 2 * hh])) * st * sr[2 * hh];
+                const float y1 = static_cast<float>(static_cast<int32_t>(rr[jb + 2 * hh + 1])) * st * sr[2 * hh + 1];
+                w[hh] = pack_bf16x2(y0, y1);
+              }
+              st_shared_v4(buf + lane * 128 + ((c16 ^ sw) << 4), w[0], w[1], w[2], w[3]);
+            }
+          } else {
+            const int sh = W4 ? 4 : 0;
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) {
+              st_shared_v4(buf + lane * 128 + ((c16 ^ sw) << 4),
+                           static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16]) >> sh),
+                           static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16 + 1]) >> sh),
+                           static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16 + 2]) >> sh),
+                           static_cast<uint32_t>(static_cast<int32_t>(r0[4 * c16 + 3]) >> sh));
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, buf, ncol0 + oc * OC, m0);
+            bulk_commit_group();
+          }
+        }
+      }
+      if (!seg.partial) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);
+      }
+      ++local;
+    }
+    if (lane == 0) bulk_wait_group<0>();  // every output store complete before exit
+  } else if (W4) {
+    // ------------------------------------------------------------ int4 unpack
+    const int ct = threadIdx.x - 32 * (2 + PAIR_EPI_WARPS);  // 0..127
+    uint32_t it = 0;
+    bool ok = true;
+    while (ok && sched.next(seg)) {
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, SITE_CONV_FULL)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = smem + s * SM::STAGE;
+        const uint8_t* packed = st + SM::A_BYTES + SM::B_BYTES;
+        uint8_t* unp = st + SM::A_BYTES;
+        for (int idx = ct; idx < 128 * 4; idx += 128) {
+          const int r = idx >> 2, pc = idx & 3;
+          const uint4 pk = *reinterpret_cast<const uint4*>(packed + r * 64 + pc * 16);
+          const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int hh = 0; hh < 4; ++hh) {
+            const uint32_t lo = (w[hh] << 4) & 0xF0F0F0F0u;
+            const uint32_t hi = w[hh] & 0xF0F0F0F0u;
+            o[2 * hh] = __byte_perm(lo, hi, 0x5140);
+            o[2 * hh + 1] = __byte_perm(lo, hi, 0x7362);
+          }
+          const int sw = r & 7;
+          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&conv[s]), 0));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no cross-CTA arrive, copy or MMA can still target either CTA
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, SM::TMEM_COLS);
+  }
+}
+
+}  // namespace convrot
