@@ -176,13 +176,12 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits);
  * Xq int8 [M, K], s_tok fp32 [M], Wq int8 [N, K], s_row fp32 [N] in;
  * Y bf16 [M, N] out.  K % 16 == 0, K <= CONVROT_MAX_K, N % 8 == 0.
  * workspace: device buffer of at least convrot_linear_workspace_bytes(M, N,
- * K, 8) bytes, zero-filled before its first use.  It holds int32 partial
- * tiles of output tiles that several CTAs share (scratch) and one arrival
- * counter per such tile; every call that returns CONVROT_OK leaves the
- * counters at zero again, so the buffer can be passed to later calls without
- * clearing, also by calls of other shapes (the counters occupy a fixed
- * region at the start of the buffer).  Calls that share one workspace must
- * not run concurrently.
+ * K, 8) bytes, zero-filled before its first use.  Output tiles whose K range
+ * is split across CTAs are summed there: one int32 accumulator and one
+ * arrival counter per such tile.  Every call that returns CONVROT_OK leaves
+ * the whole buffer zero-filled again, so it can be passed to later calls of
+ * any shape without clearing.  Calls that share one workspace must not run
+ * concurrently.
  */
 convrot_status convrot_int8_linear(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
                                    const float* s_row, int M, int N, int K, void* Y,
@@ -214,8 +213,8 @@ convrot_status convrot_w4a8_linear(const int8_t* Xq, const float* s_tok, const u
  *  - Shapes whose workspace exceeds 24 MiB are rejected with
  *    CONVROT_ERR_WORKSPACE (on a 148-SM B200 every M <= 128 fits; larger M
  *    with tiles split across CTAs does not - use convrot_int8_linear).
- *  - All calls on a device share the array: each call clears the part that
- *    must start at zero, and calls that overlap on the GPU race.
+ *  - All calls on a device share the array: each call clears the part it
+ *    uses (which must start at zero), and calls that overlap on the GPU race.
  * Arguments, layouts and return codes otherwise as convrot_int8_linear.
  */
 convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const float* s_tok, const int8_t* Wq,

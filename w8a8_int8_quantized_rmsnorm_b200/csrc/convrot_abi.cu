@@ -190,6 +190,45 @@ convrot_status launch_rowquant_pre(RowQuantArgs& a, bool rot, cudaStream_t st) {
                     : launch_rowquant_t<false, PRE, QK, false>(a, threads, st);
 }
 
+// TMA-fed activation kernel: teams of rowquant's layout, one CTA per SM, a
+// ring of stages of `rows` token rows each.
+template <bool ROT, bool NORM>
+convrot_status launch_actquant_t(ActArgs a, cudaStream_t st) {
+  auto k = actquant_kernel<ROT, NORM>;
+  const DeviceInfo d = current_device();
+  const int dyn = a.wsm_bytes + a.stages * a.rows * a.K * 2;
+  static std::atomic<int> configured[64];
+  if (d.device >= 0 && configured[d.device].load(std::memory_order_relaxed) < dyn) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+        cudaSuccess)
+      return CONVROT_ERR_CUDA;
+    configured[d.device].store(200 * 1024, std::memory_order_relaxed);
+  }
+  const int units = (a.M + a.rows - 1) / a.rows;
+  const int grid = std::max(1, std::min(units, std::max(1, d.sms)));
+  k<<<grid, 32 + a.team * a.rows, dyn, st>>>(a);
+  return launch_status();
+}
+
+// Returns false when the shape is outside what the TMA-fed kernel handles
+// (rows wider than one team of 256 threads), so the caller uses rowquant_kernel.
+bool plan_actquant(int K, ActArgs& a) {
+  const RowPlan p = plan_rows(K);
+  if (!p.resident) return false;
+  a.team = p.team;
+  // up to 12 consumer warps: several rows in flight per CTA
+  a.rows = std::max(1, 384 / p.team);
+  const int row_bytes = K * 2;
+  // keep a stage within 48 KB
+  while (a.rows > 1 && a.rows * row_bytes > 48 * 1024) --a.rows;
+  if (a.team * a.rows < 32 || (a.team * a.rows) % 32) return false;
+  a.wsm_bytes = 0;
+  const int budget = 200 * 1024;
+  const int stage = a.rows * row_bytes;
+  a.stages = std::min(ACT_MAX_STAGES, budget / stage);
+  return a.stages >= 2;
+}
+
 convrot_status check_group(int group, int K, int multiple) {
   if (group != 0 && group != 256) return CONVROT_ERR_UNSUPPORTED;
   if (K <= 0 || K > CONVROT_MAX_K) return CONVROT_ERR_SHAPE;
@@ -246,9 +285,10 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs) {
   p.sk_r = p.sk_iters % p.grid;
   // a stream-K region whose iterations split evenly into whole tiles needs no workspace
   const bool whole = p.sk_r == 0 && p.sk_q % p.num_kb == 0;
+  // one int32 accumulator tile (and one counter) per split tile and CTA
   const int ctas_per_unit = p.pair ? 2 : 1;
   p.ws_slot_bytes =
-      whole ? 0 : static_cast<size_t>(2) * p.grid * ctas_per_unit * GEMM_BM * p.bn * 4;
+      whole ? 0 : static_cast<size_t>(sk_tiles) * ctas_per_unit * GEMM_BM * p.bn * 4;
   p.ws_count_bytes = whole ? 0 : static_cast<size_t>(sk_tiles) * ctas_per_unit * 4;
   return p;
 }
@@ -317,10 +357,10 @@ convrot_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, co
   return launch_status();
 }
 
-// Workspace layout: a fixed region of tile counters at offset 0 (left at zero
-// by every successful call, whatever the shape), then the partial-tile slots.
-// Keeping the counters at a fixed place is what makes one zero-filled buffer
-// reusable across calls of different shapes.
+// Workspace layout: a fixed region of tile counters at offset 0, then one
+// int32 accumulator tile per split tile and CTA.  Every successful call leaves
+// the whole buffer zero (the finalising CTA re-zeroes its accumulator and
+// counter), so one zero-filled buffer serves calls of any shape.
 size_t ws_bytes(const GemmPlan& p) {
   if (p.ws_slot_bytes == 0) return 0;
   return kCounterBytes + p.ws_slot_bytes;
@@ -415,8 +455,8 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
   a.srow_vec = (s_row != nullptr && aligned(s_row, 16)) ? 1 : 0;
   a.out = out;
   a.ws_counts = need ? static_cast<unsigned*>(workspace) : nullptr;
-  a.ws_slots = need ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
-                    : nullptr;
+  a.ws_acc = need ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
+                  : nullptr;
   const CUtensorMap& ma = p.swap ? mw : mx;
   const CUtensorMap& mb = p.swap ? mx : mw;
   if (p.pair) {
@@ -545,6 +585,26 @@ convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
   if (!x || !Xq || !s_tok) return CONVROT_ERR_NULL;
   if (!aligned(x, 16) || !aligned(Xq, 16) || !aligned(s_tok, 4)) return CONVROT_ERR_ALIGN;
   if (norm_w && !aligned(norm_w, 16)) return CONVROT_ERR_ALIGN;
+  const bool rot = group == 256;
+  ActArgs q{};
+  q.x = static_cast<const uint16_t*>(x);
+  q.norm_w = norm_w;
+  q.xq = Xq;
+  q.s_tok = s_tok;
+  q.M = M;
+  q.K = K;
+  q.eps = eps;
+  if (plan_actquant(K, q)) {
+    if (norm_w) {
+      q.wsm_bytes = (K * 4 + 1023) / 1024 * 1024;
+      q.stages = std::min(ACT_MAX_STAGES, (200 * 1024 - q.wsm_bytes) / (q.rows * K * 2));
+    }
+    if (q.stages >= 2) {
+      cudaStream_t st = as_cuda(stream);
+      if (rot) return norm_w ? launch_actquant_t<true, true>(q, st) : launch_actquant_t<true, false>(q, st);
+      return norm_w ? launch_actquant_t<false, true>(q, st) : launch_actquant_t<false, false>(q, st);
+    }
+  }
   RowQuantArgs a{};
   a.src = static_cast<const uint16_t*>(x);
   a.vec = norm_w;
@@ -553,7 +613,6 @@ convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
   a.rows = M;
   a.K = K;
   a.eps = eps;
-  const bool rot = group == 256;
   return norm_w ? launch_rowquant_pre<PRE_NORM, QK_INT8>(a, rot, as_cuda(stream))
                 : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, rot, as_cuda(stream));
 }
@@ -666,9 +725,9 @@ convrot_status convrot_w4a8_gemm_s32(const int8_t* Xq, const uint8_t* Wq4, int M
 // the device address is looked up with cudaGetSymbolAddress once per device
 // (the first call on a device does that set-up; make that first call before
 // any stream capture).  All calls on a device share the array and it keeps the
-// last call's contents: each call clears the tile counters that must start at
-// zero, and calls that overlap on the GPU (other streams, other threads) race
-// on it.
+// last call's contents: each call clears the counters and accumulators it
+// uses, which must start at zero, and calls that overlap on the GPU (other
+// streams, other threads) race on it.
 // ===========================================================================
 constexpr size_t kStaticWorkspaceBytes = static_cast<size_t>(24) << 20;  // 24 MiB per device
 static __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
@@ -710,8 +769,8 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
   if (need > 0) {
     const convrot_status a = static_workspace_address(d.device, &ws);
     if (a != CONVROT_OK) return a;
-    if (cudaMemsetAsync(ws, 0, kCounterBytes, as_cuda(stream)) != cudaSuccess)
-      return CONVROT_ERR_CUDA;
+    // the counters and accumulators this call uses must start at zero
+    if (cudaMemsetAsync(ws, 0, need, as_cuda(stream)) != cudaSuccess) return CONVROT_ERR_CUDA;
   }
   return run_gemm(Xq, Wq, false, s_tok, s_row, M, N, K, Y, false, ws,
                   need > 0 ? kStaticWorkspaceBytes : 0, as_cuda(stream));

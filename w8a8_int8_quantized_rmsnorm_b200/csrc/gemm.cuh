@@ -45,6 +45,7 @@ constexpr int GEMM_BK = 128;  // int8 elements (bytes) of K per stage
 constexpr int GEMM_UMMA_K = 32;
 constexpr int GEMM_MAX_STAGES = 16;
 constexpr int GEMM_GROUP_A = 8;
+constexpr int GEMM_PREFETCH_AHEAD = 8;  // L2 prefetch this many K steps beyond the ring
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
 
@@ -66,8 +67,8 @@ struct GemmArgs {
   const float* s_row;
   int srow_vec;  // s_row is 16-byte aligned: vector loads in the epilogue
   void* out;
-  int32_t* ws_slots;     // [2 * gridDim.x][BM * BN] partial tiles
-  unsigned* ws_counts;   // [num_tiles - dp_tiles]
+  int32_t* ws_acc;       // [split tiles][CTAs per unit][BM * BN] int32 accumulators
+  unsigned* ws_counts;   // [split tiles][CTAs per unit] arrival counters
 };
 
 struct Segment {
@@ -149,8 +150,9 @@ struct GemmSmem {
   static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
   static constexpr int P_BYTES = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 weight tile
   static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
-  // non-swap epilogue: per epilogue warp two 4 KB staging buffers (32 rows x 128 B)
-  static constexpr int STAGING = SWAP ? 0 : 4 * 2 * 4096;
+  // per epilogue warp two 4 KB staging buffers (32 rows x 128 B) for output
+  // stores and split-tile reductions
+  static constexpr int STAGING = 4 * 2 * 4096;
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;  // TMEM columns per accumulator buffer
   static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
   static constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
@@ -233,9 +235,23 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
       }
       uint32_t it = 0;
       bool ok = true;
+      // L2 prefetch distance in K steps: beyond what the shared ring holds, so
+      // that tiles first touched in DRAM are in L2 when their load is issued
+      const int pfd = S + GEMM_PREFETCH_AHEAD;
+      auto prefetch = [&](int ta, int tb, int kb) {
+        if (W4 && SWAP)
+          tma_prefetch_l2_2d(&tmA, kb * (GEMM_BK / 2), ta * GEMM_BM);
+        else
+          tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
+        if (W4 && !SWAP)
+          tma_prefetch_l2_2d(&tmB, kb * (GEMM_BK / 2), tb * BN);
+        else
+          tma_prefetch_l2_2d(&tmB, kb * GEMM_BK, tb * BN);
+      };
       while (ok && sched.next(seg)) {
         int ta, tb;
         tile_coords(a, seg.tile, ta, tb);
+        for (int kb = seg.kb0 + S; kb < min(seg.kb1, seg.kb0 + pfd); ++kb) prefetch(ta, tb, kb);
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
@@ -243,6 +259,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
             ok = false;
             break;
           }
+          if (kb + pfd < seg.kb1) prefetch(ta, tb, kb + pfd);
           uint8_t* st = smem + s * SM::STAGE;
           mbar_arrive_expect_tx(&full[s], tx);
           if (W4 && SWAP)
@@ -334,10 +351,13 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * SM::ACC_STRIDE;
       const int arow = ta * GEMM_BM + 32 * q + lane;  // operand-A row of this thread
 
+      // A split tile: every contributing CTA adds its int32 partial into the
+      // tile's accumulator (bulk reductions performed at L2); the CTA that
+      // completes the tile's count reads it back, re-zeroes it and writes the
+      // output.
+      const int u_sk = seg.tile - a.dp_tiles;
+      int32_t* acc_tile = a.ws_acc + static_cast<size_t>(u_sk) * (GEMM_BM * BN);
       if (seg.partial) {
-        // write this CTA's partial tile to its slot: for each 32-column chunk c
-        // and warp q, 8 x 16 bytes per lane, consecutive lanes consecutive
-        int32_t* slot = a.ws_slots + static_cast<size_t>(seg.slot) * (GEMM_BM * BN);
 #pragma unroll 1
         for (int c = 0; c < BN / CW; ++c) {
           uint32_t r[32];
@@ -347,29 +367,39 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
             tmem_ld_32x32b_x16(tbase + c * CW, r);
           }
           tmem_ld_wait();
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous bulk op has read the buffer
+          __syncwarp();
 #pragma unroll
-          for (int j4 = 0; j4 < CW / 4; ++j4) {
-            uint4* dst = reinterpret_cast<uint4*>(slot) + ((c * 4 + q) * (CW / 4) + j4) * 32 + lane;
-            *dst = make_uint4(r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+          for (int j4 = 0; j4 < CW / 4; ++j4)
+            st_shared_v4(stage_buf + (j4 * 32 + lane) * 16, r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2],
+                         r[4 * j4 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            bulk_reduce_add_s32(acc_tile + (c * 4 + q) * 32 * CW, stage_buf, 128 * CW);
+            bulk_commit_group();
           }
         }
       }
-      // the accumulator buffer can be reused once a partial tile is saved
-      // (a full tile keeps it until its output is written, below)
       bool finalize = !seg.partial;
       if (seg.partial) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tmem_empty[b]);
+        if (lane == 0) {
+          bulk_wait_group<0>();  // this warp's reductions are performed
+          fence_proxy_async_global();
+        }
+        __syncwarp();
         __threadfence();
         if (!epi_rendezvous()) break;
         if (et == 0) {
-          const int u = seg.tile - a.dp_tiles;
-          const int c_lo = sk_owner(a, u * a.num_kb);
-          const int c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
-          const unsigned prev = atomicAdd(&a.ws_counts[u], 1u);
+          const int c_lo = sk_owner(a, u_sk * a.num_kb);
+          const int c_hi = sk_owner(a, (u_sk + 1) * a.num_kb - 1);
+          __threadfence();
+          const unsigned prev = atomicAdd(&a.ws_counts[u_sk], 1u);
           const bool last = prev + 1u == static_cast<unsigned>(c_hi - c_lo + 1);
-          if (last) a.ws_counts[u] = 0u;  // leave the workspace clean for the next call
+          if (last) a.ws_counts[u_sk] = 0u;  // leave the workspace clean for the next call
           *last_flag = last ? 1 : 0;
         }
         if (!epi_rendezvous()) break;
@@ -377,12 +407,6 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
         if (finalize) __threadfence();
       }
       if (finalize) {
-        int c_lo = 0, c_hi = -1, u = 0;
-        if (seg.partial) {
-          u = seg.tile - a.dp_tiles;
-          c_lo = sk_owner(a, u * a.num_kb);
-          c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
-        }
         if (!SWAP) {
           // ---- rows of the output tile: staged through shared memory, TMA stores
           const int m = arow;
@@ -397,34 +421,29 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
               if (OC == 64) tmem_ld_32x32b_x32(tbase + oc * OC + 32, r1);
               tmem_ld_wait();
             } else {
+              // the tile's sum; leave the accumulator at zero for the next call
+              const int c0 = oc * (OC / 32);
+              uint4* base = reinterpret_cast<uint4*>(acc_tile);
+              uint4 v0[8], v1[8];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                r0[j] = 0u;
-                r1[j] = 0u;
+              for (int j4 = 0; j4 < 8; ++j4) {
+                v0[j4] = __ldcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane);
+                if (OC == 64) v1[j4] = __ldcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane);
               }
-              for (int cc = c_lo; cc <= c_hi; ++cc) {
-                const int slot_id = 2 * cc + (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
-                const uint4* base = reinterpret_cast<const uint4*>(
-                    a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN));
-                const int c0 = oc * (OC / 32);
-                uint4 v0[8], v1[8];
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                  v0[j4] = __ldcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane);
-                  if (OC == 64) v1[j4] = __ldcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane);
-                }
-#pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                  r0[4 * j4] += v0[j4].x;
-                  r0[4 * j4 + 1] += v0[j4].y;
-                  r0[4 * j4 + 2] += v0[j4].z;
-                  r0[4 * j4 + 3] += v0[j4].w;
-                  if (OC == 64) {
-                    r1[4 * j4] += v1[j4].x;
-                    r1[4 * j4 + 1] += v1[j4].y;
-                    r1[4 * j4 + 2] += v1[j4].z;
-                    r1[4 * j4 + 3] += v1[j4].w;
-                  }
+              for (int j4 = 0; j4 < 8; ++j4) {
+                __stcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane, z);
+                if (OC == 64) __stcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane, z);
+                r0[4 * j4] = v0[j4].x;
+                r0[4 * j4 + 1] = v0[j4].y;
+                r0[4 * j4 + 2] = v0[j4].z;
+                r0[4 * j4 + 3] = v0[j4].w;
+                if (OC == 64) {
+                  r1[4 * j4] = v1[j4].x;
+                  r1[4 * j4 + 1] = v1[j4].y;
+                  r1[4 * j4 + 2] = v1[j4].z;
+                  r1[4 * j4 + 3] = v1[j4].w;
                 }
               }
             }
@@ -497,23 +516,18 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
               }
               tmem_ld_wait();
             } else {
+              uint4* base = reinterpret_cast<uint4*>(acc_tile) + (c * 4 + q) * (CW / 4) * 32 + lane;
+              uint4 v[CW / 4];
 #pragma unroll
-              for (int j = 0; j < CW; ++j) r[j] = 0u;
-              for (int cc = c_lo; cc <= c_hi; ++cc) {
-                const int slot_id = 2 * cc + (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
-                const uint4* src = reinterpret_cast<const uint4*>(
-                                       a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN)) +
-                                   (c * 4 + q) * (CW / 4) * 32 + lane;
-                uint4 v[CW / 4];
+              for (int j4 = 0; j4 < CW / 4; ++j4) v[j4] = __ldcg(base + j4 * 32);
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                for (int j4 = 0; j4 < CW / 4; ++j4) v[j4] = __ldcg(src + j4 * 32);
-#pragma unroll
-                for (int j4 = 0; j4 < CW / 4; ++j4) {
-                  r[4 * j4] += v[j4].x;
-                  r[4 * j4 + 1] += v[j4].y;
-                  r[4 * j4 + 2] += v[j4].z;
-                  r[4 * j4 + 3] += v[j4].w;
-                }
+              for (int j4 = 0; j4 < CW / 4; ++j4) {
+                __stcg(base + j4 * 32, z);
+                r[4 * j4] = v[j4].x;
+                r[4 * j4 + 1] = v[j4].y;
+                r[4 * j4 + 2] = v[j4].z;
+                r[4 * j4 + 3] = v[j4].w;
               }
             }
             const int m0 = tb * BN + c * CW;
@@ -589,6 +603,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
     }
   }
 
+  __syncwarp();  // roles ran on single lanes: reconverge before the aligned barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -116,11 +116,17 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
       const uint64_t pol_b = policy_evict_first();
       uint32_t it = 0;
       bool ok = true;
+      const int pfd = S + GEMM_PREFETCH_AHEAD;
       while (ok && sched.next(seg)) {
         int ta, tb;
         tile_coords(a, seg.tile, ta, tb);
         const int arow = ta * 256 + static_cast<int>(rank) * 128;
         const int brow = tb * BN + static_cast<int>(rank) * 128;
+        auto prefetch = [&](int kb) {
+          tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, arow);
+          tma_prefetch_l2_2d(&tmB, W4 ? kb * (GEMM_BK / 2) : kb * GEMM_BK, brow);
+        };
+        for (int kb = seg.kb0 + S; kb < min(seg.kb1, seg.kb0 + pfd); ++kb) prefetch(kb);
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
@@ -128,6 +134,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
             ok = false;
             break;
           }
+          if (kb + pfd < seg.kb1) prefetch(kb + pfd);
           uint8_t* st = smem + s * SM::STAGE;
           if (W4) {
             // each CTA converts its own weight rows: completion on its own barrier
@@ -225,19 +232,30 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * BN + h * 128;
       const uint32_t lead_tmem_empty = mapa_shared(smem_addr(&tmem_empty[b]), 0);
 
+      // A split tile: every contributing pair adds its int32 partial into one
+      // accumulator per CTA of the tile (bulk reductions performed at L2); the
+      // pair that completes the tile's count reads it back, re-zeroes it and
+      // writes the output.
+      const int u_sk = seg.tile - a.dp_tiles;
+      int32_t* acc_tile = a.ws_acc + static_cast<size_t>(2 * u_sk + rank) * (GEMM_BM * BN);
       if (seg.partial) {
-        int32_t* slot = a.ws_slots + static_cast<size_t>(2 * (2 * sched.cta + rank) + (seg.slot & 1)) *
-                                         (GEMM_BM * BN);
 #pragma unroll 1
         for (int cl = 0; cl < 4; ++cl) {  // this warp's 32-column chunks
           const int c = h * 4 + cl;
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + cl * 32, r);
           tmem_ld_wait();
+          if (lane == 0) bulk_wait_group_read<0>();  // the previous reduction has read buf
+          __syncwarp();
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            uint4* dst = reinterpret_cast<uint4*>(slot) + ((c * 4 + q) * 8 + j4) * 32 + lane;
-            *dst = make_uint4(r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+          for (int j4 = 0; j4 < 8; ++j4)
+            st_shared_v4(buf + (j4 * 32 + lane) * 16, r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2],
+                         r[4 * j4 + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            bulk_reduce_add_s32(acc_tile + (c * 4 + q) * 1024, buf, 4096);
+            bulk_commit_group();
           }
         }
       }
@@ -246,15 +264,20 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);
+        if (lane == 0) {
+          bulk_wait_group<0>();  // this warp's reductions are performed
+          fence_proxy_async_global();
+        }
+        __syncwarp();
         __threadfence();
         if (!epi_rendezvous()) break;
         if (ew == 0 && lane == 0) {
-          const int u = seg.tile - a.dp_tiles;
-          const int c_lo = sk_owner(a, u * a.num_kb);
-          const int c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
-          const unsigned prev = atomicAdd(&a.ws_counts[2 * u + rank], 1u);
+          const int c_lo = sk_owner(a, u_sk * a.num_kb);
+          const int c_hi = sk_owner(a, (u_sk + 1) * a.num_kb - 1);
+          __threadfence();
+          const unsigned prev = atomicAdd(&a.ws_counts[2 * u_sk + rank], 1u);
           const bool last = prev + 1u == static_cast<unsigned>(c_hi - c_lo + 1);
-          if (last) a.ws_counts[2 * u + rank] = 0u;
+          if (last) a.ws_counts[2 * u_sk + rank] = 0u;
           *last_flag = last ? 1 : 0;
         }
         if (!epi_rendezvous()) break;
@@ -262,12 +285,6 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
         if (finalize) __threadfence();
       }
       if (finalize) {
-        int c_lo = 0, c_hi = -1, u = 0;
-        if (seg.partial) {
-          u = seg.tile - a.dp_tiles;
-          c_lo = sk_owner(a, u * a.num_kb);
-          c_hi = sk_owner(a, (u + 1) * a.num_kb - 1);
-        }
         const int m = m0 + lane;
         float st = 0.f;
         if (EPI == EPI_BF16 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
@@ -279,35 +296,29 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
             if (OC == 64) tmem_ld_32x32b_x32(tbase + oc * OC + 32, r1);
             tmem_ld_wait();
           } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              r0[j] = 0u;
-              r1[j] = 0u;
-            }
+            // the tile's sum; leave the accumulator at zero for the next call
             const int c0 = h * 4 + oc * (OC / 32);
-            for (int cc = c_lo; cc <= c_hi; ++cc) {
-              const int slot_id = 2 * (2 * cc + static_cast<int>(rank)) +
-                                  (sk_begin_of(a, cc) >= u * a.num_kb ? 0 : 1);
-              const uint4* base = reinterpret_cast<const uint4*>(
-                  a.ws_slots + static_cast<size_t>(slot_id) * (GEMM_BM * BN));
-              uint4 v0[8], v1[8];
+            uint4* base = reinterpret_cast<uint4*>(acc_tile);
+            uint4 v0[8], v1[8];
 #pragma unroll
-              for (int j4 = 0; j4 < 8; ++j4) {
-                v0[j4] = __ldcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane);
-                if (OC == 64) v1[j4] = __ldcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane);
-              }
+            for (int j4 = 0; j4 < 8; ++j4) {
+              v0[j4] = __ldcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane);
+              if (OC == 64) v1[j4] = __ldcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane);
+            }
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-              for (int j4 = 0; j4 < 8; ++j4) {
-                r0[4 * j4] += v0[j4].x;
-                r0[4 * j4 + 1] += v0[j4].y;
-                r0[4 * j4 + 2] += v0[j4].z;
-                r0[4 * j4 + 3] += v0[j4].w;
-                if (OC == 64) {
-                  r1[4 * j4] += v1[j4].x;
-                  r1[4 * j4 + 1] += v1[j4].y;
-                  r1[4 * j4 + 2] += v1[j4].z;
-                  r1[4 * j4 + 3] += v1[j4].w;
-                }
+            for (int j4 = 0; j4 < 8; ++j4) {
+              __stcg(base + ((c0 * 4 + q) * 8 + j4) * 32 + lane, z);
+              if (OC == 64) __stcg(base + (((c0 + 1) * 4 + q) * 8 + j4) * 32 + lane, z);
+              r0[4 * j4] = v0[j4].x;
+              r0[4 * j4 + 1] = v0[j4].y;
+              r0[4 * j4 + 2] = v0[j4].z;
+              r0[4 * j4 + 3] = v0[j4].w;
+              if (OC == 64) {
+                r1[4 * j4] = v1[j4].x;
+                r1[4 * j4 + 1] = v1[j4].y;
+                r1[4 * j4 + 2] = v1[j4].z;
+                r1[4 * j4 + 3] = v1[j4].w;
               }
             }
           }
@@ -411,6 +422,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     }
   }
 
+  __syncwarp();  // roles ran on single lanes: reconverge before the aligned barrier
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no cross-CTA arrive, copy or MMA can still target either CTA
