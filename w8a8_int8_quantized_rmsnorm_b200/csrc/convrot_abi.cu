@@ -259,10 +259,10 @@ int pick_bn_swap(int M) {
 
 // `units` is the number of co-resident work units: SMs for the single-CTA
 // kernel, CTA pairs (clusters of two) for the pair kernel.
-GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs) {
+GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4) {
   GemmPlan p{};
   p.swap = M <= 128;
-  p.pair = M > 256 && pairs > 0;
+  p.pair = !p.swap && pairs > 0;
   p.bn = p.swap ? pick_bn_swap(M) : 256;
   const int rowsA = p.swap ? N : M;
   const int rowsB = p.swap ? M : N;
@@ -270,7 +270,8 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs) {
   p.tilesA = (rowsA + tileA - 1) / tileA;
   p.tilesB = (rowsB + p.bn - 1) / p.bn;
   p.num_tiles = p.tilesA * p.tilesB;
-  p.num_kb = (K + GEMM_BK - 1) / GEMM_BK;
+  const int stage_k = GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
+  p.num_kb = (K + stage_k - 1) / stage_k;
   const long long total = static_cast<long long>(p.num_tiles) * p.num_kb;
   const int units = p.pair ? pairs : sms;
   // at most 2 * units tiles are split (each with one counter per CTA of the
@@ -409,7 +410,7 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const GemmPlan p = plan_gemm(M, N, K, d.sms, pair_units_for(w4, s32_out, d.device));
+  const GemmPlan p = plan_gemm(M, N, K, d.sms, pair_units_for(w4, s32_out, d.device), w4);
   const size_t need = ws_bytes(p);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CONVROT_ERR_WORKSPACE;
   if (need > 0 && !aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
@@ -647,7 +648,7 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return 0;
   // the bf16 and int32 outputs share the schedule, so either plan gives the size
-  return ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(weight_bits == 4, false, d.device)));
+  return ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(weight_bits == 4, false, d.device), weight_bits == 4));
 }
 
 static convrot_status linear_common(const int8_t* Xq, const float* s_tok, const void* Wq,
@@ -763,7 +764,7 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
     return CONVROT_ERR_ALIGN;
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(false, false, d.device)));
+  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(false, false, d.device), false));
   if (need > kStaticWorkspaceBytes) return CONVROT_ERR_WORKSPACE;  // shape too large for the array
   void* ws = nullptr;
   if (need > 0) {

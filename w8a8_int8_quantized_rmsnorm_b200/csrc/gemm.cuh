@@ -7,8 +7,9 @@
 // "Matmul" row; the int4 weight layout of "MossInt4", "Format".)
 //
 // Kernel structure (one CTA per SM, persistent):
-//   warp 0      TMA producer: int8 tiles of both operands, 128 bytes of K per
-//               stage, 128-byte swizzle, into a ring of shared-memory stages;
+//   warp 0      TMA producer: int8 tiles of both operands, one or two 128-byte
+//               K atoms per stage, 128-byte swizzle, into a ring of
+//               shared-memory stages;
 //   warp 1      allocates TMEM and issues tcgen05.mma kind::i8 (one thread),
 //               128 x BN x 32 per instruction, s32 accumulators in TMEM,
 //               two accumulator buffers so the epilogue of one tile overlaps
@@ -28,12 +29,14 @@
 //
 // Work split.  Output tiles are ordered in groups of 8 A-tiles for L2 reuse.
 // Whole waves of tiles are handed out round-robin (data-parallel).  The last
-// one to two waves are split evenly by K-block over all CTAs (stream-K).  A
-// CTA whose range covers only part of a tile writes its int32 partial tile to
-// its own workspace slot, then increments the tile's counter; the CTA that
-// brings the counter to the number of contributors sums all partial slots in
-// a fixed order (deterministic), writes the output and resets the counter.
-// No CTA ever waits on another CTA.
+// one to two waves are split evenly by pipeline stage over all CTAs
+// (stream-K).  A CTA whose range covers only part of a tile adds its int32
+// partial tile into the tile's accumulator in the workspace (bulk add
+// reductions performed at L2), then increments the tile's counter; the CTA
+// that brings the counter to the number of contributors reads the sum back,
+// re-zeroes the accumulator and the counter, and writes the output.  Integer
+// addition makes the result independent of arrival order.  No CTA ever waits
+// on another CTA.
 #pragma once
 
 #include "ptx.cuh"
@@ -41,11 +44,21 @@
 namespace convrot {
 
 constexpr int GEMM_BM = 128;
-constexpr int GEMM_BK = 128;  // int8 elements (bytes) of K per stage
+constexpr int GEMM_BK = 128;  // int8 elements (bytes) of K per swizzle atom
 constexpr int GEMM_UMMA_K = 32;
 constexpr int GEMM_MAX_STAGES = 16;
 constexpr int GEMM_GROUP_A = 8;
-constexpr int GEMM_PREFETCH_AHEAD = 8;  // L2 prefetch this many K steps beyond the ring
+constexpr int GEMM_PREFETCH_ATOMS = 8;  // L2 prefetch this many K atoms beyond the ring
+// 128-byte K atoms per pipeline stage.  A single thread issues every
+// tcgen05.mma, and each MMA issue, stage wait and commit costs that thread tens
+// of cycles: with one atom (four 32-deep MMAs) per stage the issuing thread
+// needs more than the 512 tensor-pipe cycles of a 128 x 256 x 128 (or pair
+// 256 x 256 x 128) step and the pipe idles between steps.  Two atoms per stage
+// halve the waits and commits per MMA.  Int4 weights keep one atom: their
+// stage also holds the packed tile, and unpacking sets their pace.
+__host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
+  return w4 ? 1 : ((pair || swap) ? 2 : 1);
+}
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
 
@@ -58,7 +71,7 @@ struct GemmArgs {
   int rowsA, rowsB;  // rows of operands A and B
   int tilesA, tilesB;
   int num_tiles;
-  int num_kb;
+  int num_kb;        // pipeline stages of K per tile (KA atoms of 128 bytes each)
   int stages;
   int dp_tiles;      // tiles [0, dp_tiles) are data-parallel
   int sk_iters;      // (num_tiles - dp_tiles) * num_kb
@@ -145,10 +158,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Shared-memory plan (offsets from a 1024-byte aligned base).
 template <int BN, bool W4, bool SWAP>
 struct GemmSmem {
-  static constexpr int A_BYTES = GEMM_BM * GEMM_BK;
-  static constexpr int B_BYTES = BN * GEMM_BK;
+  static constexpr int KA = gemm_katoms(W4, false, SWAP);
+  static constexpr int A_ATOM = GEMM_BM * GEMM_BK;  // one 128-byte K atom of the A tile
+  static constexpr int B_ATOM = BN * GEMM_BK;
+  static constexpr int A_BYTES = KA * A_ATOM;
+  static constexpr int B_BYTES = KA * B_ATOM;
   static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
   static constexpr int P_BYTES = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 weight tile
+  static_assert(!W4 || KA == 1, "int4 stages hold one K atom");
   static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
   // per epilogue warp two 4 KB staging buffers (32 rows x 128 B) for output
   // stores and split-tile reductions
@@ -237,21 +254,27 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
       bool ok = true;
       // L2 prefetch distance in K steps: beyond what the shared ring holds, so
       // that tiles first touched in DRAM are in L2 when their load is issued
-      const int pfd = S + GEMM_PREFETCH_AHEAD;
+      constexpr int KA = SM::KA;
+      const int pfd = S + GEMM_PREFETCH_ATOMS / KA;
       auto prefetch = [&](int ta, int tb, int kb) {
-        if (W4 && SWAP)
-          tma_prefetch_l2_2d(&tmA, kb * (GEMM_BK / 2), ta * GEMM_BM);
-        else
-          tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
-        if (W4 && !SWAP)
-          tma_prefetch_l2_2d(&tmB, kb * (GEMM_BK / 2), tb * BN);
-        else
-          tma_prefetch_l2_2d(&tmB, kb * GEMM_BK, tb * BN);
+#pragma unroll
+        for (int j = 0; j < KA; ++j) {
+          const int k0 = (kb * KA + j) * GEMM_BK;
+          if (W4 && SWAP)
+            tma_prefetch_l2_2d(&tmA, k0 / 2, ta * GEMM_BM);
+          else
+            tma_prefetch_l2_2d(&tmA, k0, ta * GEMM_BM);
+          if (W4 && !SWAP)
+            tma_prefetch_l2_2d(&tmB, k0 / 2, tb * BN);
+          else
+            tma_prefetch_l2_2d(&tmB, k0, tb * BN);
+        }
       };
       while (ok && sched.next(seg)) {
         int ta, tb;
         tile_coords(a, seg.tile, ta, tb);
-        for (int kb = seg.kb0 + S; kb < min(seg.kb1, seg.kb0 + pfd); ++kb) prefetch(ta, tb, kb);
+        // the first ring-full of loads goes out before the initial prefetch window
+        const int win = min(seg.kb1, seg.kb0 + S) - 1;
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
@@ -259,19 +282,25 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
             ok = false;
             break;
           }
-          if (kb + pfd < seg.kb1) prefetch(ta, tb, kb + pfd);
           uint8_t* st = smem + s * SM::STAGE;
           mbar_arrive_expect_tx(&full[s], tx);
-          if (W4 && SWAP)
-            tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmA, &full[s], kb * (GEMM_BK / 2),
-                        ta * GEMM_BM, pol_a);
-          else
-            tma_load_2d(st, &tmA, &full[s], kb * GEMM_BK, ta * GEMM_BM, pol_a);
-          if (W4 && !SWAP)
-            tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], kb * (GEMM_BK / 2),
-                        tb * BN, pol_b);
-          else
-            tma_load_2d(st + SM::A_BYTES, &tmB, &full[s], kb * GEMM_BK, tb * BN, pol_b);
+#pragma unroll
+          for (int j = 0; j < KA; ++j) {
+            // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
+            const int k0 = (kb * KA + j) * GEMM_BK;
+            if (W4 && SWAP)
+              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmA, &full[s], k0 / 2, ta * GEMM_BM,
+                          pol_a);
+            else
+              tma_load_2d(st + j * SM::A_ATOM, &tmA, &full[s], k0, ta * GEMM_BM, pol_a);
+            if (W4 && !SWAP)
+              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], k0 / 2, tb * BN, pol_b);
+            else
+              tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, &full[s], k0, tb * BN, pol_b);
+          }
+          if (kb + pfd < seg.kb1) prefetch(ta, tb, kb + pfd);
+          if (kb == win)
+            for (int kp = seg.kb0 + S; kp < min(seg.kb1, seg.kb0 + pfd); ++kp) prefetch(ta, tb, kp);
         }
       }
       // drain: make sure no copy is still landing in shared memory when the CTA exits
@@ -305,9 +334,13 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
           const uint32_t sa = smem_addr(smem + s * SM::STAGE);
           const uint32_t sb = sa + SM::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
-            mma_s8(d, sw128_kmajor_desc(sa + k * GEMM_UMMA_K), sw128_kmajor_desc(sb + k * GEMM_UMMA_K),
-                   IDESC, (kb > seg.kb0 || k > 0) ? 1u : 0u);
+          for (int j = 0; j < SM::KA; ++j) {
+#pragma unroll
+            for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
+              mma_s8(d, sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K),
+                     sw128_kmajor_desc(sb + j * SM::B_ATOM + k * GEMM_UMMA_K), IDESC,
+                     (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u);
+            }
           }
           mma_commit(&empty[s]);
         }

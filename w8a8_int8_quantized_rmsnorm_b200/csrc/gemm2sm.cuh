@@ -1,4 +1,4 @@
-// W8A8 / W4A8 ConvRot linear on CTA pairs (tcgen05 cta_group::2), for M > 256.
+// W8A8 / W4A8 ConvRot linear on CTA pairs (tcgen05 cta_group::2), for M > 128.
 //
 // Same arithmetic as gemm_kernel ("MOSS-Image Qwen3.5-9B text encoder, INT8
 // (W8A8, ConvRot)", file table, "Matmul" row; int4 layout of "MossInt4",
@@ -7,9 +7,10 @@
 //
 // Two CTAs of a cluster share one 256 x 256 output tile.  Each CTA stages its
 // own 128 rows of activations (A) and its own 128 rows of weights (B, half of
-// the tile's N) - 32 KB per 128-byte K step instead of the 48 KB one CTA needs
-// for a 128 x 256 tile - so six stages fit and each SM pulls 64 B/clk at the
-// tensor pipe's rate.  One thread of the leader CTA issues
+// the tile's N) - 32 KB per 128-byte K atom instead of the 48 KB one CTA needs
+// for a 128 x 256 tile - so each SM pulls 64 B/clk at the tensor pipe's rate.
+// An int8 stage holds two K atoms (64 KB, three stages): eight MMAs per stage
+// wait and commit keep the single issuing thread ahead of the tensor pipe.  One thread of the leader CTA issues
 // tcgen05.mma.cta_group::2 (256 x 256 x 32 int8): the hardware reads A and B
 // from both CTAs' shared memory and writes each CTA's 128 accumulator rows x
 // 256 columns into that CTA's TMEM.  TMA loads never use cluster multicast:
@@ -34,9 +35,13 @@ constexpr int PAIR_EPI_WARPS = 8;
 
 template <bool W4>
 struct Gemm2Smem {
-  static constexpr int A_BYTES = 128 * GEMM_BK;
-  static constexpr int B_BYTES = 128 * GEMM_BK;
+  static constexpr int KA = gemm_katoms(W4, true, false);
+  static constexpr int A_ATOM = 128 * GEMM_BK;  // this CTA's 128 rows x one 128-byte K atom
+  static constexpr int B_ATOM = 128 * GEMM_BK;
+  static constexpr int A_BYTES = KA * A_ATOM;
+  static constexpr int B_BYTES = KA * B_ATOM;
   static constexpr int P_BYTES = W4 ? 128 * (GEMM_BK / 2) : 0;
+  static_assert(!W4 || KA == 1, "int4 stages hold one K atom");
   static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
   static constexpr int STAGING = PAIR_EPI_WARPS * 4096;
   static constexpr int TMEM_COLS = 512;
@@ -116,17 +121,22 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
       const uint64_t pol_b = policy_evict_first();
       uint32_t it = 0;
       bool ok = true;
-      const int pfd = S + GEMM_PREFETCH_AHEAD;
+      const int pfd = S + GEMM_PREFETCH_ATOMS / SM::KA;
       while (ok && sched.next(seg)) {
         int ta, tb;
         tile_coords(a, seg.tile, ta, tb);
         const int arow = ta * 256 + static_cast<int>(rank) * 128;
         const int brow = tb * BN + static_cast<int>(rank) * 128;
         auto prefetch = [&](int kb) {
-          tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, arow);
-          tma_prefetch_l2_2d(&tmB, W4 ? kb * (GEMM_BK / 2) : kb * GEMM_BK, brow);
+#pragma unroll
+          for (int j = 0; j < SM::KA; ++j) {
+            const int k0 = (kb * SM::KA + j) * GEMM_BK;
+            tma_prefetch_l2_2d(&tmA, k0, arow);
+            tma_prefetch_l2_2d(&tmB, W4 ? k0 / 2 : k0, brow);
+          }
         };
-        for (int kb = seg.kb0 + S; kb < min(seg.kb1, seg.kb0 + pfd); ++kb) prefetch(kb);
+        // the first ring-full of loads goes out before the initial prefetch window
+        const int win = min(seg.kb1, seg.kb0 + S) - 1;
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
@@ -134,7 +144,6 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
             ok = false;
             break;
           }
-          if (kb + pfd < seg.kb1) prefetch(kb + pfd);
           uint8_t* st = smem + s * SM::STAGE;
           if (W4) {
             // each CTA converts its own weight rows: completion on its own barrier
@@ -146,9 +155,17 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
             // both CTAs' tiles complete on the leader's barrier, which the leader arms
             const uint32_t lead_full = mapa_shared(smem_addr(&full[s]), 0);
             if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (SM::A_BYTES + SM::B_BYTES));
-            tma_load_2d_pair(st, &tmA, lead_full, kb * GEMM_BK, arow, pol_a);
-            tma_load_2d_pair(st + SM::A_BYTES, &tmB, lead_full, kb * GEMM_BK, brow, pol_b);
+#pragma unroll
+            for (int j = 0; j < SM::KA; ++j) {
+              // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
+              const int k0 = (kb * SM::KA + j) * GEMM_BK;
+              tma_load_2d_pair(st + j * SM::A_ATOM, &tmA, lead_full, k0, arow, pol_a);
+              tma_load_2d_pair(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, lead_full, k0, brow, pol_b);
+            }
           }
+          if (kb + pfd < seg.kb1) prefetch(kb + pfd);
+          if (kb == win)
+            for (int kp = seg.kb0 + S; kp < min(seg.kb1, seg.kb0 + pfd); ++kp) prefetch(kp);
         }
       }
       if (W4) {
@@ -185,10 +202,13 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
           const uint32_t sa = smem_addr(smem + s * SM::STAGE);
           const uint32_t sb = sa + SM::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
-            mma_s8_pair(d, sw128_kmajor_desc(sa + k * GEMM_UMMA_K),
-                        sw128_kmajor_desc(sb + k * GEMM_UMMA_K), IDESC,
-                        (kb > seg.kb0 || k > 0) ? 1u : 0u);
+          for (int j = 0; j < SM::KA; ++j) {
+#pragma unroll
+            for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
+              mma_s8_pair(d, sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K),
+                          sw128_kmajor_desc(sb + j * SM::B_ATOM + k * GEMM_UMMA_K), IDESC,
+                          (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u);
+            }
           }
           mma_commit_pair_mc(&empty[s], 0x3);
         }

@@ -424,8 +424,9 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
 // The other warps form R teams of T = (padded) K/64 threads; team r takes row r
 // of a stage, reads its 64 elements per thread from shared memory in the same
 // lane layout as rowquant_kernel, releases the stage at once, and runs the
-// same transform, reductions and 16-byte code stores.  The RMSNorm multiplier
-// 1 + w is computed once per CTA into shared memory.
+// 256-point FWHT in packed f32x2 arithmetic (lane bits by shuffles), the row
+// reductions and 8-byte code stores.  The RMSNorm weight w is bulk-copied once
+// per CTA into shared memory together with the first rows.
 // ---------------------------------------------------------------------------
 constexpr int ACT_MAX_STAGES = 8;
 
@@ -534,7 +535,8 @@ __device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(stat
 
 // Lane (g, L) of a 256-group holds elements 32i + 8L + r (i, r = 0..7) as 32
 // pairs: pair p = 4i + r/2 holds (r even, r odd).  Loads them from a staged
-// row in shared memory, accumulates sum(x^2) and applies the norm multiplier.
+// row in shared memory, accumulates sum(x^2) and applies the norm multiplier
+// 1 + w (wsm holds w).
 template <bool NORM>
 __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm, int K, int g,
                                           int L, bool ok, uint64_t (&v)[32], float& sq) {
@@ -559,10 +561,11 @@ __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm
         m0 = *reinterpret_cast<const ulonglong2*>(wsm + e);
         m1 = *reinterpret_cast<const ulonglong2*>(wsm + e + 4);
       }
-      v[4 * i] = f2_mul(v[4 * i], m0.x);
-      v[4 * i + 1] = f2_mul(v[4 * i + 1], m0.y);
-      v[4 * i + 2] = f2_mul(v[4 * i + 2], m1.x);
-      v[4 * i + 3] = f2_mul(v[4 * i + 3], m1.y);
+      // x * (1 + w) as x + x * w: one rounding of the exact product
+      v[4 * i] = f2_fma(v[4 * i], m0.x, v[4 * i]);
+      v[4 * i + 1] = f2_fma(v[4 * i + 1], m0.y, v[4 * i + 1]);
+      v[4 * i + 2] = f2_fma(v[4 * i + 2], m1.x, v[4 * i + 2]);
+      v[4 * i + 3] = f2_fma(v[4 * i + 3], m1.y, v[4 * i + 3]);
     }
   }
   sq += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
@@ -641,7 +644,7 @@ template <bool ROT, bool NORM>
 __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
   __shared__ float s_max[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
   __shared__ double s_sum[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
-  __shared__ uint64_t full[ACT_MAX_STAGES], empty[ACT_MAX_STAGES];
+  __shared__ uint64_t full[ACT_MAX_STAGES], empty[ACT_MAX_STAGES], wbar;
   __shared__ int abort_word;
   extern __shared__ __align__(1024) uint8_t act_smem[];
   float* wsm = reinterpret_cast<float*>(act_smem);
@@ -658,11 +661,9 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], cwarps);
     }
+    mbar_init(&wbar, 1);
     abort_word = 0;
     fence_barrier_init();
-  }
-  if (NORM) {
-    for (int k = threadIdx.x; k < a.K; k += blockDim.x) wsm[k] = 1.0f + a.norm_w[k];
   }
   __syncthreads();
 
@@ -670,6 +671,11 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      if (NORM) {
+        // the norm weight w [K] fp32, copied once per CTA next to the first rows
+        mbar_arrive_expect_tx(&wbar, static_cast<uint32_t>(a.K) * 4u);
+        bulk_load_1d(wsm, a.norm_w, static_cast<uint32_t>(a.K) * 4u, &wbar);
+      }
       int i = 0;
       for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
         const int s = i % a.stages;
@@ -695,6 +701,10 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
         int dummy = 0;
         mbar_wait(&full[j % a.stages], (j / a.stages) & 1u, &dummy, SITE_DRAIN);
       }
+      if (NORM) {
+        int dummy = 0;
+        mbar_wait(&wbar, 0u, &dummy, SITE_DRAIN);
+      }
     }
     return;
   }
@@ -706,6 +716,7 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
   const int g = t >> 2;
   const int G = (a.K + 255) >> 8;
   TeamReducer red{s_max, s_sum, a.team, slot, lane, t >> 5, a.team >> 5, 0};
+  if (NORM && !mbar_wait(&wbar, 0u, abort_flag, SITE_EPI_FULL)) return;
   int i = 0;
   for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
     const int s = i % a.stages;
