@@ -32,11 +32,14 @@ def _rand_scales(n, seed):
 
 
 SHAPES = [
-    # (M, N, K): operand roles swap at M <= 128
+    # (M, N, K): operand roles swap at M <= 128; above it CTA pairs take
+    # 256 x 256 tiles, a single wave of at most one tile per four-CTA cluster
+    # splits K over two pairs, larger grids split by stream-K
     (1, 256, 512), (3, 136, 512), (16, 1024, 4096), (17, 264, 1040), (40, 512, 256),
     (64, 128, 768), (100, 2056, 144), (128, 520, 4096),
     (129, 264, 512), (256, 512, 4096), (300, 1032, 1040), (512, 4096, 12288),
     (1024, 1024, 4096), (2048, 1536, 16), (777, 8, 32),
+    (1280, 2560, 1088), (2048, 4096, 1024),
 ]
 
 
@@ -114,10 +117,11 @@ def test_w4a8_linear_bf16(cr, M, N, K):
 
 
 def test_workspace_reuse_and_determinism(cr):
-    # this shape splits tiles by K across CTAs, so partial tiles meet in the
-    # workspace; reusing it for further calls only gives the right answer if
-    # every call restores the tile counters to zero
-    M, N, K = 512, 4096, 12288
+    # this shape (48 pair tiles, more than fit as split-K clusters) splits
+    # tiles by K across CTA pairs, so partial tiles meet in the workspace;
+    # reusing it for further calls only gives the right answer if every call
+    # restores the tile counters and accumulators to zero
+    M, N, K = 768, 4096, 8192
     assert cr.convrot_linear_workspace_bytes(M, N, K, 8) > 0
     ws = cr.Workspace()
     X = _rand_i8((M, K), 11)
@@ -135,8 +139,8 @@ def test_workspace_reuse_and_determinism(cr):
 def test_workspace_shared_across_shapes(cr):
     # one buffer, calls of different shapes and operand roles in a row
     ws = cr.Workspace()
-    for (M, N, K) in [(512, 4096, 12288), (1, 24576, 4096), (129, 264, 512), (2048, 1024, 4096),
-                      (16, 1024, 4096), (512, 4096, 12288)]:
+    for (M, N, K) in [(768, 4096, 8192), (1, 24576, 4096), (129, 264, 512), (2048, 1024, 4096),
+                      (512, 4096, 12288), (16, 1024, 4096), (768, 4096, 8192)]:
         X = _rand_i8((M, K), M + N)
         W = _rand_i8((N, K), N + K)
         acc = cr.convrot_int8_gemm_s32(X.cuda(), W.cuda(), workspace=ws)
@@ -145,7 +149,8 @@ def test_workspace_shared_across_shapes(cr):
 
 
 def test_workspace_too_small_is_rejected(cr):
-    M, N, K = 512, 4096, 12288
+    M, N, K = 768, 4096, 8192
+    assert cr.convrot_linear_workspace_bytes(M, N, K, 8) > 0
     X = torch.zeros(M, K, dtype=torch.int8, device="cuda")
     W = torch.zeros(N, K, dtype=torch.int8, device="cuda")
     s = torch.ones(max(M, N), device="cuda")

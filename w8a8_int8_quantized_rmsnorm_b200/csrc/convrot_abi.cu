@@ -242,7 +242,8 @@ constexpr size_t kCounterBytes = 4096;
 
 struct GemmPlan {
   bool swap;
-  bool pair;  // CTA-pair kernel (256-row tiles); grid/units below count pairs
+  bool pair;   // CTA-pair kernel (256-row tiles); grid/units below count pairs
+  bool split;  // pair kernel in split-K clusters of two pairs; grid counts clusters
   int bn;
   int tilesA, tilesB, num_tiles, num_kb;
   int grid;
@@ -259,7 +260,9 @@ int pick_bn_swap(int M) {
 
 // `units` is the number of co-resident work units: SMs for the single-CTA
 // kernel, CTA pairs (clusters of two) for the pair kernel.
-GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4) {
+// `clusters4` is the number of co-resident four-CTA clusters of the split
+// pair kernel (0 if unavailable).
+GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int clusters4) {
   GemmPlan p{};
   p.swap = M <= 128;
   p.pair = !p.swap && pairs > 0;
@@ -272,6 +275,17 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4) {
   p.num_tiles = p.tilesA * p.tilesB;
   const int stage_k = GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
   p.num_kb = (K + stage_k - 1) / stage_k;
+  // One wave of 256 x 256 tiles that fits the co-resident clusters: each tile
+  // is split in two K halves over two CTA pairs whose partial sums meet in
+  // shared memory (no stream-K workspace, no L2 round trip).
+  if (p.pair && !w4 && clusters4 > 0 && p.num_kb >= 2 && p.num_tiles <= clusters4) {
+    p.split = true;
+    p.grid = p.num_tiles;
+    p.dp_tiles = 0;
+    p.sk_iters = p.sk_q = p.sk_r = 0;
+    p.ws_slot_bytes = p.ws_count_bytes = 0;
+    return p;
+  }
   const long long total = static_cast<long long>(p.num_tiles) * p.num_kb;
   const int units = p.pair ? pairs : sms;
   // at most 2 * units tiles are split (each with one counter per CTA of the
@@ -328,28 +342,70 @@ int pair_units(int device) {
   return clusters;
 }
 
+// Co-resident clusters of four CTAs of the split pair kernel (once per device).
+template <int EPI>
+int split_units(int device) {
+  static std::atomic<int> cached[64];
+  if (device < 0 || device >= 64) return 0;
+  int v = cached[device].load(std::memory_order_relaxed);
+  if (v != 0) return v;
+  using SM = Gemm2Smem<false>;
+  auto k = gemm2sm_kernel<false, EPI, true>;
+  const int avail = 227 * 1024 - 1024 - SM::total(0);
+  const int stages = std::max(2, std::min(GEMM_MAX_STAGES, avail / SM::STAGE));
+  const int smem = SM::total(stages) + 1024;
+  int clusters = 0;
+  if (stages * SM::STAGE >= SPLIT_RECV_BYTES &&
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(4, 1, 1);
+    cfg.blockDim = dim3(320, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 4;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&clusters, k, &cfg) != cudaSuccess) clusters = 0;
+  }
+  cudaGetLastError();
+  if (clusters <= 0) clusters = -1;  // split mode unavailable
+  cached[device].store(clusters, std::memory_order_relaxed);
+  return clusters;
+}
+
+int split_units_for(bool w4, bool s32, int device) {
+  if (w4) return 0;
+  const int c = s32 ? split_units<EPI_S32>(device) : split_units<EPI_BF16>(device);
+  return c > 0 ? c : 0;
+}
+
 int pair_units_for(bool w4, bool s32, int device) {
   if (w4) return s32 ? pair_units<true, EPI_S32>(device) : pair_units<true, EPI_BF16>(device);
   return s32 ? pair_units<false, EPI_S32>(device) : pair_units<false, EPI_BF16>(device);
 }
 
-template <bool W4, int EPI>
+// `units` counts CTA pairs, or (SPLIT) clusters of two pairs.
+template <bool W4, int EPI, bool SPLIT = false>
 convrot_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
-                                GemmArgs a, int pairs, cudaStream_t st) {
+                                GemmArgs a, int units, cudaStream_t st) {
   using SM = Gemm2Smem<W4>;
-  auto k = gemm2sm_kernel<W4, EPI>;
+  auto k = gemm2sm_kernel<W4, EPI, SPLIT>;
   const int avail = 227 * 1024 - 1024 - SM::total(0);
   const int stages = std::max(2, std::min(GEMM_MAX_STAGES, avail / SM::STAGE));
   a.stages = stages;
   const int smem = SM::total(stages) + 1024;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  const int cluster = SPLIT ? 4 : 2;
+  cfg.gridDim = dim3(cluster * units, 1, 1);
   cfg.blockDim = dim3(W4 ? 448 : 320, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.x = cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -410,7 +466,8 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const GemmPlan p = plan_gemm(M, N, K, d.sms, pair_units_for(w4, s32_out, d.device), w4);
+  const GemmPlan p = plan_gemm(M, N, K, d.sms, pair_units_for(w4, s32_out, d.device), w4,
+                                split_units_for(w4, s32_out, d.device));
   const size_t need = ws_bytes(p);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CONVROT_ERR_WORKSPACE;
   if (need > 0 && !aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
@@ -460,6 +517,9 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
                   : nullptr;
   const CUtensorMap& ma = p.swap ? mw : mx;
   const CUtensorMap& mb = p.swap ? mx : mw;
+  if (p.split)
+    return s32_out ? launch_gemm_pair<false, EPI_S32, true>(ma, mb, my, a, p.grid, st)
+                   : launch_gemm_pair<false, EPI_BF16, true>(ma, mb, my, a, p.grid, st);
   if (p.pair) {
     if (w4)
       return s32_out ? launch_gemm_pair<true, EPI_S32>(ma, mb, my, a, p.grid, st)
@@ -648,7 +708,8 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return 0;
   // the bf16 and int32 outputs share the schedule, so either plan gives the size
-  return ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(weight_bits == 4, false, d.device), weight_bits == 4));
+  return ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(weight_bits == 4, false, d.device), weight_bits == 4,
+                            split_units_for(weight_bits == 4, false, d.device)));
 }
 
 static convrot_status linear_common(const int8_t* Xq, const float* s_tok, const void* Wq,
@@ -764,7 +825,8 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
     return CONVROT_ERR_ALIGN;
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(false, false, d.device), false));
+  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(false, false, d.device), false,
+                            split_units_for(false, false, d.device)));
   if (need > kStaticWorkspaceBytes) return CONVROT_ERR_WORKSPACE;  // shape too large for the array
   void* ws = nullptr;
   if (need > 0) {

@@ -64,7 +64,7 @@ constexpr int EPI_S32 = 1;
 
 // wait sites recorded in the device error word
 constexpr unsigned SITE_PROD_EMPTY = 1, SITE_MMA_FULL = 2, SITE_MMA_TMEM = 3, SITE_EPI_FULL = 4,
-                   SITE_CONV_FULL = 5, SITE_DRAIN = 6, SITE_EPI_SYNC = 7;
+                   SITE_CONV_FULL = 5, SITE_DRAIN = 6, SITE_EPI_SYNC = 7, SITE_SPLIT = 8;
 
 struct GemmArgs {
   int M, N, K;

@@ -10,7 +10,8 @@
 // the tile's N) - 32 KB per 128-byte K atom instead of the 48 KB one CTA needs
 // for a 128 x 256 tile - so each SM pulls 64 B/clk at the tensor pipe's rate.
 // An int8 stage holds two K atoms (64 KB, three stages): eight MMAs per stage
-// wait and commit keep the single issuing thread ahead of the tensor pipe.  One thread of the leader CTA issues
+// wait and commit keep the single issuing thread ahead of the tensor pipe.
+// One thread of the leader CTA issues
 // tcgen05.mma.cta_group::2 (256 x 256 x 32 int8): the hardware reads A and B
 // from both CTAs' shared memory and writes each CTA's 128 accumulator rows x
 // 256 columns into that CTA's TMEM.  TMA loads never use cluster multicast:
@@ -25,6 +26,15 @@
 // Work split, stream-K partial tiles and their workspace protocol are those of
 // gemm_kernel with a CTA pair as the unit; each CTA of the pair fixes up its
 // own 128 rows of a split tile.
+//
+// SPLIT (int8 weights; at most one tile per cluster): clusters of four CTAs,
+// two pairs per tile.  Pair 0 accumulates the first half of K and owns the
+// output; pair 1 accumulates the second half.  When its MMAs are complete each
+// owner CTA (its stage ring drained) arms a 128 KB receive barrier and
+// signals its partner CTA (cluster rank + 2), which reads its accumulators
+// from TMEM and writes them with st.async into the owner's stage ring; the
+// owner adds them in its epilogue.  The partial sums cross the cluster's
+// shared-memory network, not L2, and no workspace is used.
 #pragma once
 
 #include "gemm.cuh"
@@ -52,11 +62,14 @@ struct Gemm2Smem {
   }
 };
 
-template <bool W4, int EPI>
+constexpr int SPLIT_RECV_BYTES = 128 * 128 * 4;  // half of one CTA's accumulator columns
+
+template <bool W4, int EPI, bool SPLIT = false>
 __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = Gemm2Smem<W4>;
+  static_assert(!(SPLIT && W4), "the split-K cluster mode is int8 only");
   constexpr int BN = 256;
   constexpr uint32_t IDESC = idesc_s8s8s32(256, BN);
 
@@ -71,13 +84,19 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
   uint64_t* tmem_empty = tmem_full + 2;
   uint64_t* drain = tmem_empty + 2;
   uint64_t* epi_sync = drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 1);
+  uint64_t* recv = epi_sync + 1;   // SPLIT owner: the partner's partial has landed
+  uint64_t* ready = epi_sync + 2;  // SPLIT partner: the owner's stage ring is free
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t rank = crank & 1u;    // role in the CTA pair: 0 = leader
+  const uint32_t lead = crank & ~1u;   // cluster rank of this pair's leader
+  const uint32_t pq = crank >> 1;      // SPLIT: 0 = owner pair, 1 = partner pair
+  const uint16_t pair_mask = static_cast<uint16_t>(0x3u << lead);
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
 
@@ -93,6 +112,8 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     }
     mbar_init(drain, 1);
     mbar_init(epi_sync, PAIR_EPI_WARPS);
+    mbar_init(recv, 1);
+    mbar_init(ready, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
@@ -106,13 +127,28 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA use
+  cluster_sync();  // barriers of every CTA initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   Schedule sched;
   sched.init(a, pair, npairs);
   Segment seg;
+  // SPLIT: cluster u takes tile u; pair pq takes half pq of its K stages
+  const int cunit = static_cast<int>(blockIdx.x >> 2);
+  bool split_taken = false;
+  auto next_seg = [&](Segment& sg) -> bool {
+    if (!SPLIT) return sched.next(sg);
+    if (split_taken || cunit >= a.num_tiles) return false;
+    split_taken = true;
+    const int half = (a.num_kb + 1) >> 1;
+    sg.tile = cunit;
+    sg.kb0 = pq ? half : 0;
+    sg.kb1 = pq ? a.num_kb : half;
+    sg.partial = false;
+    sg.slot = -1;
+    return true;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -122,7 +158,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
       uint32_t it = 0;
       bool ok = true;
       const int pfd = S + GEMM_PREFETCH_ATOMS / SM::KA;
-      while (ok && sched.next(seg)) {
+      while (ok && next_seg(seg)) {
         int ta, tb;
         tile_coords(a, seg.tile, ta, tb);
         const int arow = ta * 256 + static_cast<int>(rank) * 128;
@@ -153,7 +189,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
                         pol_b);
           } else {
             // both CTAs' tiles complete on the leader's barrier, which the leader arms
-            const uint32_t lead_full = mapa_shared(smem_addr(&full[s]), 0);
+            const uint32_t lead_full = mapa_shared(smem_addr(&full[s]), lead);
             if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (SM::A_BYTES + SM::B_BYTES));
 #pragma unroll
             for (int j = 0; j < SM::KA; ++j) {
@@ -185,7 +221,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     if (lane == 0 && rank == 0) {
       uint32_t it = 0, local = 0;
       bool ok = true;
-      while (ok && sched.next(seg)) {
+      while (ok && next_seg(seg)) {
         const uint32_t b = local & 1u;
         const uint32_t use = local >> 1;
         if (!mbar_wait(&tmem_empty[b], (use & 1u) ^ 1u, abort_flag, SITE_MMA_TMEM)) break;
@@ -210,10 +246,10 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
                           (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u);
             }
           }
-          mma_commit_pair_mc(&empty[s], 0x3);
+          mma_commit_pair_mc(&empty[s], pair_mask);
         }
         if (!ok) break;
-        mma_commit_pair_mc(&tmem_full[b], 0x3);
+        mma_commit_pair_mc(&tmem_full[b], pair_mask);
         ++local;
       }
       // every MMA this thread issued must be complete before TMEM is released
@@ -238,19 +274,72 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     };
     constexpr int OC = (EPI == EPI_BF16) ? 64 : 32;  // output columns per 128-byte staged row
     uint8_t* buf = smem + SM::staging_offset(S) + ew * 4096;
-    while (sched.next(seg)) {
+    // columns of a tile this warp finalises: its 128-column half, or in SPLIT
+    // mode 64 columns of its own pair's half of the tile
+    constexpr int FC = SPLIT ? 64 : 128;
+    while (next_seg(seg)) {
       const uint32_t b = local & 1u;
       const uint32_t use = local >> 1;
+      int ta, tb;
+      tile_coords(a, seg.tile, ta, tb);
+      const int m0 = ta * 256 + static_cast<int>(rank) * 128 + 32 * q;  // first row of this warp
+      const int fcol = SPLIT ? static_cast<int>(pq) * 128 + h * 64 : h * 128;
+      const int ncol0 = tb * BN + fcol;  // first output column this warp finalises
+      // output scales, loaded while the accumulators are still being computed:
+      // lane l holds s_row of column ncol0 + 32 c + l
+      const int m = m0 + lane;
+      float st = 0.f;
+      float srl[FC / 32];
+#pragma unroll
+      for (int c = 0; c < FC / 32; ++c) srl[c] = 0.f;
+      if (EPI == EPI_BF16) {
+        if (m < a.M) st = __ldg(a.s_tok + m) * (W4 ? 0.0625f : 1.0f);
+#pragma unroll
+        for (int c = 0; c < FC / 32; ++c) {
+          const int n = ncol0 + 32 * c + lane;
+          if (n < a.N) srl[c] = __ldg(a.s_row + n);
+        }
+      }
       const bool got = mbar_wait(&tmem_full[b], use & 1u, abort_flag, SITE_EPI_FULL);
       __syncwarp();
       if (!got) break;
       tc_fence_after();
-      int ta, tb;
-      tile_coords(a, seg.tile, ta, tb);
-      const int m0 = ta * 256 + static_cast<int>(rank) * 128 + 32 * q;  // first row of this warp
-      const int ncol0 = tb * BN + h * 128;                              // first column of this warp
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * BN + h * 128;
-      const uint32_t lead_tmem_empty = mapa_shared(smem_addr(&tmem_empty[b]), 0);
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * BN;
+      const uint32_t tbase = tq + h * 128;  // this warp's 128-column half (stream-K path)
+      const uint32_t lead_tmem_empty = mapa_shared(smem_addr(&tmem_empty[b]), lead);
+
+      // SPLIT: the CTA of the other pair with the same rows finalises the
+      // columns this warp sends, and sends the ones this warp finalises.  The
+      // receive area in the stage ring holds, per warp, its 32 rows x 64
+      // columns as 2 chunks of 32 columns, each 8 x (32 lanes x 16 bytes).
+      const uint32_t recv_off = static_cast<uint32_t>(q * 2 + h) * 8192u;
+      if (SPLIT) {
+        const uint32_t other = pq ? crank - 2u : crank + 2u;
+        if (ew == 0 && lane == 0) {
+          // this CTA's MMAs are complete, so its stage ring is free
+          mbar_arrive_expect_tx(recv, SPLIT_RECV_BYTES);
+          mbar_arrive_cluster(mapa_shared(smem_addr(ready), other));
+        }
+        const bool go = mbar_wait(ready, 0u, abort_flag, SITE_SPLIT);
+        __syncwarp();
+        if (!go) break;
+        const int scol = (1 - static_cast<int>(pq)) * 128 + h * 64;
+        const uint32_t rbar = mapa_shared(smem_addr(recv), other);
+        const uint32_t rbase = mapa_shared(smem_addr(smem), other) + recv_off;
+#pragma unroll 1
+        for (int cl = 0; cl < 2; ++cl) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tq + scol + cl * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4)
+            st_async_v4(rbase + static_cast<uint32_t>((cl * 8 + j4) * 512 + lane * 16), rbar,
+                        r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+        }
+        const bool got_partial = mbar_wait(recv, 0u, abort_flag, SITE_SPLIT);
+        __syncwarp();
+        if (!got_partial) break;
+      }
 
       // A split tile: every contributing pair adds its int32 partial into one
       // accumulator per CTA of the tile (bulk reductions performed at L2); the
@@ -305,16 +394,34 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
         if (finalize) __threadfence();
       }
       if (finalize) {
-        const int m = m0 + lane;
-        float st = 0.f;
-        if (EPI == EPI_BF16 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
-#pragma unroll 1
-        for (int oc = 0; oc < 128 / OC; ++oc) {
+#pragma unroll
+        for (int oc = 0; oc < FC / OC; ++oc) {
           uint32_t r0[32], r1[32];
           if (!seg.partial) {
-            tmem_ld_32x32b_x32(tbase + oc * OC, r0);
-            if (OC == 64) tmem_ld_32x32b_x32(tbase + oc * OC + 32, r1);
+            tmem_ld_32x32b_x32(tq + fcol + oc * OC, r0);
+            if (OC == 64) tmem_ld_32x32b_x32(tq + fcol + oc * OC + 32, r1);
             tmem_ld_wait();
+            if (SPLIT) {
+              // add the other pair's half-K partial (exact int32 sums)
+              const uint8_t* rb = smem + recv_off;
+              const int c0 = oc * (OC / 32);
+#pragma unroll
+              for (int j4 = 0; j4 < 8; ++j4) {
+                const uint4 p0 = *reinterpret_cast<const uint4*>(rb + (c0 * 8 + j4) * 512 + lane * 16);
+                r0[4 * j4] += p0.x;
+                r0[4 * j4 + 1] += p0.y;
+                r0[4 * j4 + 2] += p0.z;
+                r0[4 * j4 + 3] += p0.w;
+                if (OC == 64) {
+                  const uint4 p1 =
+                      *reinterpret_cast<const uint4*>(rb + ((c0 + 1) * 8 + j4) * 512 + lane * 16);
+                  r1[4 * j4] += p1.x;
+                  r1[4 * j4 + 1] += p1.y;
+                  r1[4 * j4 + 2] += p1.z;
+                  r1[4 * j4 + 3] += p1.w;
+                }
+              }
+            }
           } else {
             // the tile's sum; leave the accumulator at zero for the next call
             const int c0 = h * 4 + oc * (OC / 32);
@@ -346,27 +453,15 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
           __syncwarp();
           const int sw = lane & 7;
           if (EPI == EPI_BF16) {
-            const int n0 = ncol0 + oc * OC;
 #pragma unroll
             for (int c16 = 0; c16 < 8; ++c16) {
               const uint32_t* rr = c16 < 4 ? r0 : r1;
               const int jb = (c16 & 3) * 8;
-              const int n = n0 + c16 * 8;
+              // s_row of columns oc * 64 + c16 * 8 + 0..7, held by lanes jb..jb+7
+              const float srv = srl[oc * 2 + (c16 >> 2)];
               float sr[8];
-              if (n < a.N) {
-                if (a.srow_vec) {
-                  const float4 s0 = __ldg(reinterpret_cast<const float4*>(a.s_row + n));
-                  const float4 s1 = __ldg(reinterpret_cast<const float4*>(a.s_row + n + 4));
-                  sr[0] = s0.x; sr[1] = s0.y; sr[2] = s0.z; sr[3] = s0.w;
-                  sr[4] = s1.x; sr[5] = s1.y; sr[6] = s1.z; sr[7] = s1.w;
-                } else {
 #pragma unroll
-                  for (int hh = 0; hh < 8; ++hh) sr[hh] = __ldg(a.s_row + n + hh);
-                }
-              } else {
-#pragma unroll
-                for (int hh = 0; hh < 8; ++hh) sr[hh] = 0.f;
-              }
+              for (int hh = 0; hh < 8; ++hh) sr[hh] = __shfl_sync(0xffffffffu, srv, jb + hh);
               uint32_t w[4];
 #pragma unroll
               for (int hh = 0; hh < 4; ++hh) {
@@ -408,7 +503,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     const int ct = threadIdx.x - 32 * (2 + PAIR_EPI_WARPS);  // 0..127
     uint32_t it = 0;
     bool ok = true;
-    while (ok && sched.next(seg)) {
+    while (ok && next_seg(seg)) {
       for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1u;
@@ -437,7 +532,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&conv[s]), 0));
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&conv[s]), lead));
       }
     }
   }

@@ -300,6 +300,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// 16-byte store into the shared memory of another CTA of the cluster; its
+// bytes complete transactions on that CTA's barrier at `bar_cluster_addr`.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t bar_cluster_addr,
+                                            uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          cluster_addr),
+      "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster_addr)
+      : "memory");
+}
+
 // 2-D TMA load into this CTA's shared memory whose completion is counted on
 // the barrier at `bar_cluster_addr`, which may belong to the pair's leader CTA.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
