@@ -33,7 +33,11 @@
  *    (norm_w, col_scale) must be 16-byte aligned; per-row scale vectors
  *    (s_tok, s_row) 4-byte aligned; workspaces 256-byte aligned.
  *  - Work is enqueued on `stream` (NULL = legacy default stream) and runs
- *    asynchronously; no call synchronises the stream.
+ *    asynchronously; no call synchronises the stream.  The per-token kernels
+ *    (convrot_rotate_quant_act, the linears and GEMMs) are launched with
+ *    programmatic dependent launch: their set-up may overlap the end of the
+ *    previous kernel on the stream, and each waits for that kernel to
+ *    complete before it reads or writes any memory, so stream order holds.
  *  - Arguments are validated on the host before anything is enqueued; on a
  *    validation error nothing is launched.  M = 0 (or N = 0) returns
  *    CONVROT_OK without launching.  A failed launch returns CONVROT_ERR_CUDA.

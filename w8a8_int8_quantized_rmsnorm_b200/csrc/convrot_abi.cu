@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/convrot.h"
 #include "gemm.cuh"
@@ -156,6 +157,35 @@ RowPlan plan_rows(int K) {
   return p;
 }
 
+// Launches a hot-path kernel with programmatic dependent launch (its set-up
+// may overlap the tail of the previous kernel on the stream; the kernel waits
+// for that kernel before touching memory) and, if cluster > 1, in clusters.
+template <typename... KArgs, typename... Args>
+convrot_status launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  if (cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...) != cudaSuccess) return CONVROT_ERR_CUDA;
+  return launch_status();
+}
+
 template <bool ROT, int PRE, int QK, bool RES>
 convrot_status launch_rowquant_t(const RowQuantArgs& a, int threads, cudaStream_t st) {
   auto k = rowquant_kernel<ROT, PRE, QK, RES>;
@@ -171,8 +201,7 @@ convrot_status launch_rowquant_t(const RowQuantArgs& a, int threads, cudaStream_
   }
   const int row_blocks = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
   const int grid = std::max(1, std::min(row_blocks, std::max(1, per_sm) * std::max(1, d.sms)));
-  k<<<grid, threads, 0, st>>>(a);
-  return launch_status();
+  return launch_pdl(k, dim3(grid), dim3(threads), 0, st, 1, a);
 }
 
 template <int PRE, int QK>
@@ -206,8 +235,7 @@ convrot_status launch_actquant_t(ActArgs a, cudaStream_t st) {
   }
   const int units = (a.M + a.rows - 1) / a.rows;
   const int grid = std::max(1, std::min(units, std::max(1, d.sms)));
-  k<<<grid, 32 + a.team * a.rows, dyn, st>>>(a);
-  return launch_status();
+  return launch_pdl(k, dim3(grid), dim3(32 + a.team * a.rows), dyn, st, 1, a);
 }
 
 // Returns false when the shape is outside what the TMA-fed kernel handles
@@ -397,21 +425,8 @@ convrot_status launch_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb, co
   const int stages = std::max(2, std::min(GEMM_MAX_STAGES, avail / SM::STAGE));
   a.stages = stages;
   const int smem = SM::total(stages) + 1024;
-  cudaLaunchConfig_t cfg = {};
   const int cluster = SPLIT ? 4 : 2;
-  cfg.gridDim = dim3(cluster * units, 1, 1);
-  cfg.blockDim = dim3(W4 ? 448 : 320, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k, ma, mb, my, a) != cudaSuccess) return CONVROT_ERR_CUDA;
-  return launch_status();
+  return launch_pdl(k, dim3(cluster * units), dim3(W4 ? 448 : 320), smem, st, cluster, ma, mb, my, a);
 }
 
 // Workspace layout: a fixed region of tile counters at offset 0, then one
@@ -444,8 +459,7 @@ convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const
     configured_device_mask |= bit;
   }
   constexpr int threads = W4 ? 320 : 192;
-  k<<<grid, threads, smem, st>>>(ma, mb, my, a);
-  return launch_status();
+  return launch_pdl(k, dim3(grid), dim3(threads), smem, st, 1, ma, mb, my, a);
 }
 
 template <bool SWAP, bool W4, int EPI>

@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
                 const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = GemmSmem<BN, W4, SWAP>;
   constexpr int CW = SM::CW;
+  pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
   constexpr uint32_t IDESC = idesc_s8s8s32(GEMM_BM, BN);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -234,6 +235,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // operands, scales and the output may belong to the previous kernel
 
   Schedule sched;
   sched.init(a, blockIdx.x, gridDim.x);

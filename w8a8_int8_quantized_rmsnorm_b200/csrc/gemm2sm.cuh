@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
                    const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = Gemm2Smem<W4>;
   static_assert(!(SPLIT && W4), "the split-K cluster mode is int8 only");
+  pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
   constexpr int BN = 256;
   constexpr uint32_t IDESC = idesc_s8s8s32(256, BN);
 
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
   cluster_sync();  // barriers of every CTA initialised before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // operands, scales and the output may belong to the previous kernel
 
   Schedule sched;
   sched.init(a, pair, npairs);

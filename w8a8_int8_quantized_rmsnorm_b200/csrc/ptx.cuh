@@ -300,6 +300,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with it may start while
+// the previous kernel on the stream is finishing: pdl_wait() returns once
+// every kernel it depends on has completed and its writes are visible, and
+// no memory a previous kernel may write is touched before it.
+// pdl_launch_dependents() lets the next kernel be scheduled as SMs free up.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // 16-byte store into the shared memory of another CTA of the cluster; its
 // bytes complete transactions on that CTA's barrier at `bar_cluster_addr`.
 __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t bar_cluster_addr,

@@ -291,6 +291,8 @@ template <bool ROT, int PRE, int QK, bool RESIDENT>
 __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
   __shared__ float s_max[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
   __shared__ double s_sum[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
+  pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
+  pdl_wait();
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -642,6 +644,7 @@ __device__ __forceinline__ void act3_store(int8_t* row, int K, int g, int L, boo
 
 template <bool ROT, bool NORM>
 __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
+  pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
   __shared__ float s_max[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
   __shared__ double s_sum[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
   __shared__ uint64_t full[ACT_MAX_STAGES], empty[ACT_MAX_STAGES], wbar;
@@ -666,6 +669,7 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();  // x, w, Xq and s_tok may belong to the previous kernel
 
   const int units = (a.M + a.rows - 1) / a.rows;
   if (warp == 0) {
