@@ -547,7 +547,7 @@ __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm
   for (int i = 0; i < 8; ++i) {
     const int e = g * 256 + i * 32 + L * 8;
     uint4 raw = make_uint4(0, 0, 0, 0);
-    if (ok && e < K) raw = *reinterpret_cast<const uint4*>(srow + e);
+    if (ok && e < K) raw = ld_shared_v4(srow + e);
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     uint64_t acc = 0;
 #pragma unroll
@@ -560,8 +560,11 @@ __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm
     if (NORM) {
       ulonglong2 m0 = make_ulonglong2(0ull, 0ull), m1 = m0;
       if (ok && e < K) {
-        m0 = *reinterpret_cast<const ulonglong2*>(wsm + e);
-        m1 = *reinterpret_cast<const ulonglong2*>(wsm + e + 4);
+        const uint4 u0 = ld_shared_v4(wsm + e), u1 = ld_shared_v4(wsm + e + 4);
+        m0 = make_ulonglong2(u0.x | (static_cast<uint64_t>(u0.y) << 32),
+                             u0.z | (static_cast<uint64_t>(u0.w) << 32));
+        m1 = make_ulonglong2(u1.x | (static_cast<uint64_t>(u1.y) << 32),
+                             u1.z | (static_cast<uint64_t>(u1.w) << 32));
       }
       // x * (1 + w) as x + x * w: one rounding of the exact product
       v[4 * i] = f2_fma(v[4 * i], m0.x, v[4 * i]);
