@@ -54,10 +54,11 @@ constexpr int GEMM_PREFETCH_ATOMS = 8;  // L2 prefetch this many K atoms beyond 
 // of cycles: with one atom (four 32-deep MMAs) per stage the issuing thread
 // needs more than the 512 tensor-pipe cycles of a 128 x 256 x 128 (or pair
 // 256 x 256 x 128) step and the pipe idles between steps.  Two atoms per stage
-// halve the waits and commits per MMA.  Int4 weights keep one atom: their
-// stage also holds the packed tile, and unpacking sets their pace.
+// halve the waits and commits per MMA.  Int4 weights on the single-CTA
+// kernel keep one atom (its stage also holds the packed tile); the pair
+// kernel unpacks them in place and takes two.
 __host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
-  return w4 ? 1 : ((pair || swap) ? 2 : 1);
+  return w4 ? (pair ? 2 : 1) : ((pair || swap) ? 2 : 1);
 }
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;

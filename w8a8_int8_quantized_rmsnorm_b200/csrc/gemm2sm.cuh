@@ -50,9 +50,11 @@ struct Gemm2Smem {
   static constexpr int B_ATOM = 128 * GEMM_BK;
   static constexpr int A_BYTES = KA * A_ATOM;
   static constexpr int B_BYTES = KA * B_ATOM;
-  static constexpr int P_BYTES = W4 ? 128 * (GEMM_BK / 2) : 0;
-  static_assert(!W4 || KA == 1, "int4 stages hold one K atom");
-  static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+  // int4: the packed half-width tile of each K atom (128 rows x 64 bytes)
+  // lands in the upper half of that atom's B slot and is expanded in place
+  static constexpr int PACKED_OFF = B_ATOM / 2;
+  static constexpr int PACKED_ATOM = 128 * (GEMM_BK / 2);
+  static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGING = PAIR_EPI_WARPS * 4096;
   static constexpr int TMEM_COLS = 512;
   __host__ __device__ static int staging_offset(int stages) { return stages * STAGE; }
@@ -87,7 +89,8 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
   uint64_t* epi_sync = drain + 1;
   uint64_t* recv = epi_sync + 1;   // SPLIT owner: the partner's partial has landed
   uint64_t* ready = epi_sync + 2;  // SPLIT partner: the owner's stage ring is free
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 3);
+  uint64_t* cv_sync = epi_sync + 3;  // int4: rendezvous of the four converter warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -115,6 +118,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     mbar_init(epi_sync, PAIR_EPI_WARPS);
     mbar_init(recv, 1);
     mbar_init(ready, 1);
+    mbar_init(cv_sync, 4);
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
@@ -185,10 +189,14 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
           uint8_t* st = smem + s * SM::STAGE;
           if (W4) {
             // each CTA converts its own weight rows: completion on its own barrier
-            mbar_arrive_expect_tx(&full[s], SM::A_BYTES + SM::P_BYTES);
-            tma_load_2d(st, &tmA, &full[s], kb * GEMM_BK, arow, pol_a);
-            tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], kb * (GEMM_BK / 2), brow,
-                        pol_b);
+            mbar_arrive_expect_tx(&full[s], SM::A_BYTES + SM::KA * SM::PACKED_ATOM);
+#pragma unroll
+            for (int j = 0; j < SM::KA; ++j) {
+              const int k0 = (kb * SM::KA + j) * GEMM_BK;
+              tma_load_2d(st + j * SM::A_ATOM, &tmA, &full[s], k0, arow, pol_a);
+              tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM + SM::PACKED_OFF, &tmB, &full[s], k0 / 2,
+                          brow, pol_b);
+            }
           } else {
             // both CTAs' tiles complete on the leader's barrier, which the leader arms
             const uint32_t lead_full = mapa_shared(smem_addr(&full[s]), lead);
@@ -502,8 +510,11 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
     if (lane == 0) bulk_wait_group<0>();  // every output store complete before exit
   } else if (W4) {
     // ------------------------------------------------------------ int4 unpack
+    // Each thread reads its share of every packed atom of the stage (4 x 16
+    // bytes per atom), the four warps meet (bounded), then each writes the
+    // unpacked 128-byte swizzled rows, which overwrite the packed bytes.
     const int ct = threadIdx.x - 32 * (2 + PAIR_EPI_WARPS);  // 0..127
-    uint32_t it = 0;
+    uint32_t it = 0, cv_phase = 0;
     bool ok = true;
     while (ok && next_seg(seg)) {
       for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
@@ -514,23 +525,44 @@ __global__ void __launch_bounds__(W4 ? 448 : 320, 1)
           break;
         }
         uint8_t* st = smem + s * SM::STAGE;
-        const uint8_t* packed = st + SM::A_BYTES + SM::B_BYTES;
-        uint8_t* unp = st + SM::A_BYTES;
-        for (int idx = ct; idx < 128 * 4; idx += 128) {
-          const int r = idx >> 2, pc = idx & 3;
-          const uint4 pk = *reinterpret_cast<const uint4*>(packed + r * 64 + pc * 16);
-          const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
-          uint32_t o[8];
+        uint4 pk[SM::KA][4];
 #pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            const uint32_t lo = (w[hh] << 4) & 0xF0F0F0F0u;
-            const uint32_t hi = w[hh] & 0xF0F0F0F0u;
-            o[2 * hh] = __byte_perm(lo, hi, 0x5140);
-            o[2 * hh + 1] = __byte_perm(lo, hi, 0x7362);
+        for (int j = 0; j < SM::KA; ++j) {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int idx = ct + 128 * t, r = idx >> 2, pc = idx & 3;
+            pk[j][t] = ld_shared_v4(st + SM::A_BYTES + j * SM::B_ATOM + SM::PACKED_OFF + r * 64 +
+                                    pc * 16);
           }
-          const int sw = r & 7;
-          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(cv_sync);
+        const bool met = mbar_wait(cv_sync, cv_phase & 1u, abort_flag, SITE_CONV_FULL);
+        ++cv_phase;
+        __syncwarp();
+        if (!met) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int j = 0; j < SM::KA; ++j) {
+          uint8_t* unp = st + SM::A_BYTES + j * SM::B_ATOM;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int idx = ct + 128 * t, r = idx >> 2, pc = idx & 3;
+            const uint32_t w[4] = {pk[j][t].x, pk[j][t].y, pk[j][t].z, pk[j][t].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) {
+              const uint32_t lo = (w[hh] << 4) & 0xF0F0F0F0u;
+              const uint32_t hi = w[hh] & 0xF0F0F0F0u;
+              o[2 * hh] = __byte_perm(lo, hi, 0x5140);
+              o[2 * hh + 1] = __byte_perm(lo, hi, 0x7362);
+            }
+            const int sw = r & 7;
+            st_shared_v4(unp + r * 128 + (((2 * pc) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+            st_shared_v4(unp + r * 128 + (((2 * pc + 1) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
