@@ -362,16 +362,16 @@ def run_ours(args, rank, world, dev):
     # ridge (~250 tokens) and weight-stream (HBM) bound below it
     ridge_bound = "tensor" if w.M > 256 else "hbm"
     if ridge_bound == "tensor":
-        roof = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::i8)",
+        roof = {"bound": "tensor", "kernel": "W8A8/W4A8 GEMM launch (tcgen05 kind::i8)",
                 "achieved": round(k2_achieved_tops, 1), "peak": round(int8_peak, 1),
                 "unit": "TOP/s", "frac": round(k2_achieved_tops / int8_peak, 4),
                 "peak_note": f"{peaks['source']}: 2 x dense bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
     else:
-        roof = {"bound": "hbm", "kernel": "gemm_kernel (tcgen05 kind::i8)",
+        roof = {"bound": "hbm", "kernel": "W8A8/W4A8 GEMM launch (tcgen05 kind::i8)",
                 "achieved": round(k2_achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(k2_achieved_gbs / peaks["hbm_gbs"], 4),
                 "peak_note": f"{peaks['source']} copy bandwidth"}
-    roof["traffic"] = profiled_traffic("gemm_kernel", args.workload)
+    roof["traffic"] = profiled_traffic("gemm", args.workload)
     roof["algorithmic_per_launch"] = (k2_ops / n_k2) if ridge_bound == "tensor" else (k2_bytes / n_k2)
 
     result = {
@@ -406,6 +406,7 @@ def run_ours(args, rank, world, dev):
             "rotate_quant_act": {"launches_per_step": n_k1, "avg_us": round(k1_avg * 1e3, 3),
                                  "bound": "hbm", "achieved_GBps": round(k1_achieved_gbs, 1),
                                  "frac": round(k1_achieved_gbs / peaks["hbm_gbs"], 4),
+                                 "traffic": profiled_traffic("rotate_quant_act", args.workload),
                                  "algorithmic_bytes_per_step": k1_bytes},
             "gemm": {"launches_per_step": n_k2, "avg_us": round(k2_avg * 1e3, 3),
                      "achieved_TOPs": round(k2_achieved_tops, 1),
