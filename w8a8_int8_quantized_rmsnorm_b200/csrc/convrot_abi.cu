@@ -267,6 +267,7 @@ convrot_status check_group(int group, int K, int multiple) {
 
 // ------------------------------------------------------------------ GEMM plan
 constexpr size_t kCounterBytes = 4096;
+constexpr int kFixupStages = 4;
 
 struct GemmPlan {
   bool swap;
@@ -322,7 +323,19 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   p.grid = static_cast<int>(std::min<long long>(std::min(std::max(1, units), max_grid), total));
   const int waves = p.num_tiles / p.grid;
   p.dp_tiles = waves >= 2 ? (waves - 1) * p.grid : 0;
-  const int sk_tiles = p.num_tiles - p.dp_tiles;
+  int sk_tiles = p.num_tiles - p.dp_tiles;
+  // Stream-K evens out the last waves but pays for its split tiles (partial
+  // reductions and the finalising read-back, about kFixupStages stage-times).
+  // In stage units per unit: whole waves, against the data-parallel waves plus
+  // the evened-out remainder plus the fix-up.  Ties go to plain waves.
+  const long long t_dp = static_cast<long long>((p.num_tiles + p.grid - 1) / p.grid) * p.num_kb;
+  const long long sk_total = static_cast<long long>(sk_tiles) * p.num_kb;
+  const long long t_sk = static_cast<long long>(p.dp_tiles / p.grid) * p.num_kb +
+                         (sk_total + p.grid - 1) / p.grid + kFixupStages;
+  if (t_dp <= t_sk) {
+    p.dp_tiles = p.num_tiles;
+    sk_tiles = 0;
+  }
   p.sk_iters = sk_tiles * p.num_kb;
   p.sk_q = p.sk_iters / p.grid;
   p.sk_r = p.sk_iters % p.grid;

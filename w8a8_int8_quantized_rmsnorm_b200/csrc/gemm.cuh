@@ -182,8 +182,11 @@ struct GemmSmem {
   }
 };
 
+// One CTA per SM.  Registers are allocated per SM sub-partition (16K each, a
+// CTA's warps spread over four): with 6 (10) warps, two (three) share one, so
+// 255 (168) registers per thread is the most a launch can use.
 template <int BN, bool SWAP, bool W4, int EPI>
-__global__ void __launch_bounds__(W4 ? 320 : 192, 1)
+__global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = GemmSmem<BN, W4, SWAP>;

@@ -66,8 +66,11 @@ struct Gemm2Smem {
 
 constexpr int SPLIT_RECV_BYTES = 128 * 128 * 4;  // half of one CTA's accumulator columns
 
+// One CTA per SM.  Registers are allocated per SM sub-partition (16K each, a
+// CTA's warps spread over four): with 10 (14) warps, three (four) share one,
+// so 168 (128) registers per thread is the most a launch can use.
 template <bool W4, int EPI, bool SPLIT = false>
-__global__ void __launch_bounds__(W4 ? 448 : 320, 1)
+__global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
     gemm2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = Gemm2Smem<W4>;
