@@ -396,7 +396,7 @@ int split_units(int device) {
   const int stages = std::max(2, std::min(GEMM_MAX_STAGES, avail / SM::STAGE));
   const int smem = SM::total(stages) + 1024;
   int clusters = 0;
-  if (stages * SM::STAGE >= SPLIT_RECV_BYTES &&
+  if (stages * SM::STAGE >= 2 * SPLIT_RECV_BYTES &&  // receive area + send staging
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(4, 1, 1);

@@ -28,13 +28,14 @@
 // own 128 rows of a split tile.
 //
 // SPLIT (int8 weights; at most one tile per cluster): clusters of four CTAs,
-// two pairs per tile.  Pair 0 accumulates the first half of K and owns the
-// output; pair 1 accumulates the second half.  When its MMAs are complete each
-// owner CTA (its stage ring drained) arms a 128 KB receive barrier and
-// signals its partner CTA (cluster rank + 2), which reads its accumulators
-// from TMEM and writes them with st.async into the owner's stage ring; the
-// owner adds them in its epilogue.  The partial sums cross the cluster's
-// shared-memory network, not L2, and no workspace is used.
+// two pairs per tile.  Pair 0 accumulates the first half of K, pair 1 the
+// second half.  When its MMAs are complete each CTA (its stage ring drained)
+// arms a 64 KB receive barrier and tells the CTA of the other pair with the
+// same rows (cluster rank +/- 2).  Each CTA stages, in its own ring, the half
+// of its accumulator columns that the other CTA finalises and sends it with
+// one shared-to-shared bulk copy per warp; each then adds the received half to
+// its own and finalises half of the tile's columns.  The partial sums cross
+// the cluster's shared-memory network, not L2, and no workspace is used.
 #pragma once
 
 #include "gemm.cuh"
@@ -323,8 +324,9 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
 
       // SPLIT: the CTA of the other pair with the same rows finalises the
       // columns this warp sends, and sends the ones this warp finalises.  The
-      // receive area in the stage ring holds, per warp, its 32 rows x 64
-      // columns as 2 chunks of 32 columns, each 8 x (32 lanes x 16 bytes).
+      // receive area (the first 64 KB of the stage ring) holds, per warp, its
+      // 32 rows x 64 columns as 2 chunks of 32 columns, each 8 x (32 lanes x
+      // 16 bytes).
       const uint32_t recv_off = static_cast<uint32_t>(q * 2 + h) * 8192u;
       if (SPLIT) {
         const uint32_t other = pq ? crank - 2u : crank + 2u;
@@ -333,12 +335,11 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
           mbar_arrive_expect_tx(recv, SPLIT_RECV_BYTES);
           mbar_arrive_cluster(mapa_shared(smem_addr(ready), other));
         }
-        const bool go = mbar_wait(ready, 0u, abort_flag, SITE_SPLIT);
-        __syncwarp();
-        if (!go) break;
+        // stage the columns the other CTA finalises in this CTA's own ring (above
+        // the receive area), in the receive layout, then copy the warp's 8 KB in
+        // one bulk copy once the other CTA's ring is free
         const int scol = (1 - static_cast<int>(pq)) * 128 + h * 64;
-        const uint32_t rbar = mapa_shared(smem_addr(recv), other);
-        const uint32_t rbase = mapa_shared(smem_addr(smem), other) + recv_off;
+        uint8_t* sendbuf = smem + SPLIT_RECV_BYTES + recv_off;
 #pragma unroll 1
         for (int cl = 0; cl < 2; ++cl) {
           uint32_t r[32];
@@ -346,9 +347,16 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
           tmem_ld_wait();
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4)
-            st_async_v4(rbase + static_cast<uint32_t>((cl * 8 + j4) * 512 + lane * 16), rbar,
-                        r[4 * j4], r[4 * j4 + 1], r[4 * j4 + 2], r[4 * j4 + 3]);
+            st_shared_v4(sendbuf + (cl * 8 + j4) * 512 + lane * 16, r[4 * j4], r[4 * j4 + 1],
+                         r[4 * j4 + 2], r[4 * j4 + 3]);
         }
+        fence_proxy_async_smem();
+        const bool go = mbar_wait(ready, 0u, abort_flag, SITE_SPLIT);
+        __syncwarp();
+        if (!go) break;
+        if (lane == 0)
+          bulk_copy_to_cluster(mapa_shared(smem_addr(smem), other) + recv_off, sendbuf, 8192u,
+                               mapa_shared(smem_addr(recv), other));
         const bool got_partial = mbar_wait(recv, 0u, abort_flag, SITE_SPLIT);
         __syncwarp();
         if (!got_partial) break;

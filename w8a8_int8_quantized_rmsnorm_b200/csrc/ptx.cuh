@@ -320,14 +320,15 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// 16-byte store into the shared memory of another CTA of the cluster; its
-// bytes complete transactions on that CTA's barrier at `bar_cluster_addr`.
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t bar_cluster_addr,
-                                            uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into the
+// shared memory of another CTA of the cluster, completing on that CTA's
+// barrier at `bar_cluster_addr` (no multicast; no global memory involved).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster_addr, const void* src,
+                                                     uint32_t bytes, uint32_t bar_cluster_addr) {
   asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-          cluster_addr),
-      "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster_addr)
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster_addr),
+      "r"(smem_addr(src)), "r"(bytes), "r"(bar_cluster_addr)
       : "memory");
 }
 
