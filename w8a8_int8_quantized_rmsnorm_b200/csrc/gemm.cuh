@@ -601,8 +601,9 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
       }
       ++local;
     }
-    // every output store must be complete before the CTA exits
-    if (!SWAP && lane == 0) bulk_wait_group<0>();
+    // the staged outputs must have been read before the CTA exits; the global
+    // writes themselves complete before the grid does
+    if (!SWAP && lane == 0) bulk_wait_group_read<0>();
   } else if (W4) {
     // ------------------------------------------------------------ int4 unpack
     const int ct = threadIdx.x - 192;  // 0..127

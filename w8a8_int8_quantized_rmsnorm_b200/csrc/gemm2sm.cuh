@@ -518,7 +518,9 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
       }
       ++local;
     }
-    if (lane == 0) bulk_wait_group<0>();  // every output store complete before exit
+    // the staged outputs must have been read before the CTA exits; the global
+    // writes themselves complete before the grid does
+    if (lane == 0) bulk_wait_group_read<0>();
   } else if (W4) {
     // ------------------------------------------------------------ int4 unpack
     // Each thread reads its share of every packed atom of the stage (4 x 16
