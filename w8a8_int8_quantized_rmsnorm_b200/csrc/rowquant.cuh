@@ -539,15 +539,17 @@ __device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(stat
 // pairs: pair p = 4i + r/2 holds (r even, r odd).  Loads them from a staged
 // row in shared memory, accumulates sum(x^2) and applies the norm multiplier
 // 1 + w (wsm holds w).
-template <bool NORM>
+// WHOLE: K is a multiple of 256, so a lane whose group exists is in range.
+template <bool NORM, bool WHOLE>
 __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm, int K, int g,
                                           int L, bool ok, uint64_t (&v)[32], float& sq) {
   float part[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int e = g * 256 + i * 32 + L * 8;
+    const bool in = WHOLE ? ok : (ok && e < K);
     uint4 raw = make_uint4(0, 0, 0, 0);
-    if (ok && e < K) raw = ld_shared_v4(srow + e);
+    if (in) raw = ld_shared_v4(srow + e);
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
     uint64_t acc = 0;
 #pragma unroll
@@ -559,7 +561,7 @@ __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm
     part[i] = f2_lo(acc) + f2_hi(acc);
     if (NORM) {
       ulonglong2 m0 = make_ulonglong2(0ull, 0ull), m1 = m0;
-      if (ok && e < K) {
+      if (in) {
         const uint4 u0 = ld_shared_v4(wsm + e), u1 = ld_shared_v4(wsm + e + 4);
         m0 = make_ulonglong2(u0.x | (static_cast<uint64_t>(u0.y) << 32),
                              u0.z | (static_cast<uint64_t>(u0.w) << 32));
@@ -624,6 +626,7 @@ __device__ __forceinline__ float act3_absmax(const uint64_t (&v)[32]) {
 }
 
 // int8 codes rint(v * inv) (one rounding, half-even), 8 bytes per i.
+template <bool WHOLE>
 __device__ __forceinline__ void act3_store(int8_t* row, int K, int g, int L, bool ok,
                                            const uint64_t (&v)[32], float inv) {
   const uint64_t inv2 = f2_pack(inv, inv);
@@ -640,7 +643,7 @@ __device__ __forceinline__ void act3_store(int8_t* row, int K, int g, int L, boo
     const uint32_t w0 = pack4_bytes(q[0], q[1], q[2], q[3]);
     const uint32_t w1 = pack4_bytes(q[4], q[5], q[6], q[7]);
     const int e = g * 256 + i * 32 + L * 8;
-    if (ok && e < K)
+    if (WHOLE ? ok : (ok && e < K))
       asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(row + e), "r"(w0), "r"(w1) : "memory");
   }
 }
@@ -738,7 +741,7 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
         reinterpret_cast<const uint16_t*>(ring + s * stage_bytes) + static_cast<size_t>(slot) * a.K;
     uint64_t v[32];
     float sq = 0.f;
-    act3_load<NORM>(srow, wsm, a.K, g, L, row_ok && g < G, v, sq);
+    act3_load<NORM, ROT>(srow, wsm, a.K, g, L, row_ok && g < G, v, sq);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);  // stage read: the producer may refill it
     if (ROT) act3_fwht(v, lane);
@@ -762,8 +765,8 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
     const float inv = amax > 0.f ? 127.0f / amax : 0.0f;
     if (row_ok && t == 0)
       a.s_tok[row] = amax > 0.f ? static_cast<float>(static_cast<double>(amax) * rowfac / 127.0) : 0.0f;
-    act3_store(a.xq + static_cast<size_t>(row_ok ? row : 0) * a.K, a.K, g, L, row_ok && g < G, v,
-               inv);
+    act3_store<ROT>(a.xq + static_cast<size_t>(row_ok ? row : 0) * a.K, a.K, g, L, row_ok && g < G,
+                    v, inv);
   }
 }
 
