@@ -88,6 +88,18 @@ const char* convrot_status_string(convrot_status st);
  */
 convrot_status convrot_device_status(convrot_stream_t stream, uint32_t* detail);
 
+/*
+ * Diagnostic (no counterpart on the pages): the failure path of the bounded
+ * waits, exercised without a fault.  Enqueues one small kernel whose mbarrier
+ * wait is made to run out (nothing arrives on the barrier); after about
+ * `limit_cycles` SM cycles the wait records a timeout in the device error word
+ * (bit 0, wait site 15 in bits 8..15) and the kernel returns.  A following
+ * convrot_device_status reports CONVROT_ERR_DEVICE_TIMEOUT with that detail.
+ * limit_cycles must lie in [1000, 100000000] (else CONVROT_ERR_SHAPE, nothing
+ * launched); the kernel may run up to ~1.5 ms longer than the limit.
+ */
+convrot_status convrot_selftest_wait_timeout(uint32_t limit_cycles, convrot_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * Offline weight preparation (not on the per-token path).
  * ------------------------------------------------------------------------ */

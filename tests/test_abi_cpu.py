@@ -79,6 +79,10 @@ def test_validation_before_any_launch(lib):
     # int4 clip grid
     assert lib.convrot_quantize_weight_w4(A, 4, 512, 256, None, 0.8, 1.0, 0, A, A, None) == 2
     assert lib.convrot_quantize_weight_w4(A, 4, 512, 256, None, 1.0, 0.8, 21, A, A, None) == 2
+    # the wait-timeout self-test validates its bound before launching
+    assert lib.convrot_selftest_wait_timeout(0, None) == 2
+    assert lib.convrot_selftest_wait_timeout(999, None) == 2
+    assert lib.convrot_selftest_wait_timeout(100000001, None) == 2
     # calibration may not fold in place
     assert lib.convrot_smoothquant_calibrate(A, 4, 512, A, 1e-6, A, 8, 0.5, A, A, None) == 4
 

@@ -34,6 +34,7 @@ SIGNATURES = {
     "convrot_version": (c_int, []),
     "convrot_status_string": (c_char_p, [c_int]),
     "convrot_device_status": (c_int, [c_void_p, c_uint32_p]),
+    "convrot_selftest_wait_timeout": (c_int, [ctypes.c_uint32, c_void_p]),
     "convrot_quantize_weight": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                         c_void_p, c_void_p]),
     "convrot_quantize_weight_w4": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_float,

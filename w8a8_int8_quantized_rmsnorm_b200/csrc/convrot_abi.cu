@@ -17,6 +17,7 @@
 #include "gemm.cuh"
 #include "gemm2sm.cuh"
 #include "rowquant.cuh"
+#include "selftest.cuh"
 
 using namespace convrot;
 
@@ -605,6 +606,12 @@ convrot_status convrot_device_status(convrot_stream_t stream, uint32_t* detail) 
     return CONVROT_ERR_CUDA;
   if (detail) *detail = v;
   return v ? CONVROT_ERR_DEVICE_TIMEOUT : CONVROT_OK;
+}
+
+convrot_status convrot_selftest_wait_timeout(uint32_t limit_cycles, convrot_stream_t stream) {
+  if (limit_cycles < 1000u || limit_cycles > 100000000u) return CONVROT_ERR_SHAPE;
+  selftest_wait_timeout_kernel<<<1, 32, 0, as_cuda(stream)>>>(static_cast<long long>(limit_cycles));
+  return launch_status();
 }
 
 convrot_status convrot_quantize_weight(const void* W, int N, int K, int group,

@@ -76,22 +76,28 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parit
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and
-// raises *abort) if the wait runs out, or if another role raised *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned site) {
+// raises *abort) if the wait runs out after `limit` cycles, or if another role
+// raised *abort.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                unsigned site, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long start = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (clock64() - start > WAIT_LIMIT_CYCLES) {
+      if (clock64() - start > limit) {
         report_error(ERR_WAIT_TIMEOUT | ((site & 0xFFu) << 8));
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned site) {
+  return mbar_wait_limit(bar, parity, abort, site, WAIT_LIMIT_CYCLES);
 }
 
 // ---------------------------------------------------------------- TMA
