@@ -116,12 +116,16 @@ def test_w4a8_linear_bf16(cr, M, N, K):
     assert np.all(np.abs(got - yb) <= _tol.bf16_ulp(y64) * 1.0001)
 
 
-def test_workspace_reuse_and_determinism(cr):
-    # this shape (48 pair tiles, more than fit as split-K clusters) splits
-    # tiles by K across CTA pairs, so partial tiles meet in the workspace;
-    # reusing it for further calls only gives the right answer if every call
-    # restores the tile counters and accumulators to zero
-    M, N, K = 768, 4096, 8192
+# Shapes whose plan splits tiles by K (stream-K), so partial tiles meet in the
+# workspace: a 16-token swap-kernel GEMM, and 75 pair tiles on 74 CTA pairs
+# with long K.
+STREAM_K_SHAPES = [(16, 4096, 12288), (768, 6400, 12288)]
+
+
+@pytest.mark.parametrize("M,N,K", STREAM_K_SHAPES)
+def test_workspace_reuse_and_determinism(cr, M, N, K):
+    # reusing the workspace for further calls only gives the right answer if
+    # every call restores the tile counters and accumulators to zero
     assert cr.convrot_linear_workspace_bytes(M, N, K, 8) > 0
     ws = cr.Workspace()
     X = _rand_i8((M, K), 11)
@@ -139,8 +143,8 @@ def test_workspace_reuse_and_determinism(cr):
 def test_workspace_shared_across_shapes(cr):
     # one buffer, calls of different shapes and operand roles in a row
     ws = cr.Workspace()
-    for (M, N, K) in [(768, 4096, 8192), (1, 24576, 4096), (129, 264, 512), (2048, 1024, 4096),
-                      (512, 4096, 12288), (16, 1024, 4096), (768, 4096, 8192)]:
+    for (M, N, K) in [(16, 4096, 12288), (1, 24576, 4096), (129, 264, 512), (2048, 1024, 4096),
+                      (512, 4096, 12288), (16, 1024, 4096), (768, 4096, 8192), (16, 4096, 12288)]:
         X = _rand_i8((M, K), M + N)
         W = _rand_i8((N, K), N + K)
         acc = cr.convrot_int8_gemm_s32(X.cuda(), W.cuda(), workspace=ws)
@@ -149,7 +153,7 @@ def test_workspace_shared_across_shapes(cr):
 
 
 def test_workspace_too_small_is_rejected(cr):
-    M, N, K = 768, 4096, 8192
+    M, N, K = STREAM_K_SHAPES[0]
     assert cr.convrot_linear_workspace_bytes(M, N, K, 8) > 0
     X = torch.zeros(M, K, dtype=torch.int8, device="cuda")
     W = torch.zeros(N, K, dtype=torch.int8, device="cuda")

@@ -268,7 +268,13 @@ convrot_status check_group(int group, int K, int multiple) {
 
 // ------------------------------------------------------------------ GEMM plan
 constexpr size_t kCounterBytes = 4096;
-constexpr int kFixupStages = 4;
+
+// Cost of stream-K's fix-up (partial-tile reductions at L2 and the finalising
+// read-back) in stage-times, measured against plain waves on B200: small
+// partial tiles (the token-tile of the swap kernel up to 64 wide, <= 32 KB per
+// CTA) cost about six stages; 128- and 256-wide tiles (64-128 KB per CTA) so
+// much more that plain waves won on every such shape measured.
+int fixup_stages(bool swap, int bn) { return (swap && bn <= 64) ? 6 : 24; }
 
 struct GemmPlan {
   bool swap;
@@ -326,13 +332,13 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   p.dp_tiles = waves >= 2 ? (waves - 1) * p.grid : 0;
   int sk_tiles = p.num_tiles - p.dp_tiles;
   // Stream-K evens out the last waves but pays for its split tiles (partial
-  // reductions and the finalising read-back, about kFixupStages stage-times).
+  // reductions and the finalising read-back, fixup_stages() stage-times).
   // In stage units per unit: whole waves, against the data-parallel waves plus
   // the evened-out remainder plus the fix-up.  Ties go to plain waves.
   const long long t_dp = static_cast<long long>((p.num_tiles + p.grid - 1) / p.grid) * p.num_kb;
   const long long sk_total = static_cast<long long>(sk_tiles) * p.num_kb;
   const long long t_sk = static_cast<long long>(p.dp_tiles / p.grid) * p.num_kb +
-                         (sk_total + p.grid - 1) / p.grid + kFixupStages;
+                         (sk_total + p.grid - 1) / p.grid + fixup_stages(p.swap, p.bn);
   if (t_dp <= t_sk) {
     p.dp_tiles = p.num_tiles;
     sk_tiles = 0;
