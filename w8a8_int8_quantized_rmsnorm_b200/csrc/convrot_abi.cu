@@ -519,12 +519,18 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
     if (!make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK, true)) return CONVROT_ERR_CUDA;
   }
 
-  // output map for the non-swap epilogue's TMA stores: rows of 128 bytes
+  // output map for the epilogues' TMA stores
   CUtensorMap my;
   std::memset(&my, 0, sizeof(my));
   if (!p.swap) {
     const bool ok = s32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_INT32, 32, 32, true)
                             : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, 64, true);
+    if (!ok) return CONVROT_ERR_CUDA;
+  } else {
+    // swapped roles: chunks of up to 32 tokens x 128 output columns, unswizzled
+    const uint32_t cw = bn < 32 ? bn : 32;
+    const bool ok = s32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_INT32, cw, 128, false)
+                            : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cw, 128, false);
     if (!ok) return CONVROT_ERR_CUDA;
   }
 

@@ -15,7 +15,8 @@
 //               two accumulator buffers so the epilogue of one tile overlaps
 //               the main loop of the next;
 //   warps 2-5   epilogue: tcgen05.ld of the accumulators, dequantisation to
-//               bf16 (or raw int32), global stores;
+//               bf16 (or raw int32), staged in shared memory in the output's
+//               layout and written with TMA stores;
 //   warps 6-9   (int4 weights only) unpack two signed nibbles per byte into
 //               the swizzled int8 stage the MMA reads.  A nibble n is written
 //               as the byte n * 16 (the nibble in the high half), so the MMA
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (!SWAP) tma_prefetch_desc(&tmY);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, SM::TMEM_COLS);
@@ -541,9 +542,19 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
             sbuf ^= 1;
           }
         } else {
-          // ---- swapped roles: lanes are weight rows n, columns are tokens m;
-          // for each token the warp writes 32 consecutive outputs (64 bytes)
+          // ---- swapped roles: lanes are weight rows n, columns are tokens m.
+          // Each chunk of CW tokens is staged as [CW tokens][128 columns] (the
+          // output's own layout) by the four warps, then one thread stores it
+          // with TMA.  Chunks alternate between two 16 KB halves of the staging
+          // area; before the warps meet after staging chunk k, the storing
+          // thread waits until the store of chunk k - 1 has read its half, so
+          // chunk k + 1 may overwrite it.
+          constexpr int ES = (EPI == EPI_BF16) ? 2 : 4;
           const int n = arow;
+          const int nl = 32 * q + lane;  // column of this lane in the staged tile
+          float sr = 0.f;
+          if (EPI == EPI_BF16 && n < a.N) sr = a.s_row[n] * (W4 ? 0.0625f : 1.0f);
+          bool staged_ok = true;
 #pragma unroll 1
           for (int c = 0; c < BN / CW; ++c) {
             uint32_t r[32];
@@ -570,28 +581,38 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
               }
             }
             const int m0 = tb * BN + c * CW;
-            if (n < a.N) {
+            uint8_t* xb = smem + SM::staging_offset(S) + sbuf * 16384;
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+              uint8_t* dst = xb + j * (128 * ES) + nl * ES;
               if (EPI == EPI_BF16) {
-                const float sr = a.s_row[n] * (W4 ? 0.0625f : 1.0f);
-                __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(a.out);
-#pragma unroll
-                for (int j = 0; j < CW; ++j) {
-                  const int m = m0 + j;
-                  if (m < a.M) {
-                    const float v = static_cast<float>(static_cast<int32_t>(r[j])) * __ldg(a.s_tok + m) * sr;
-                    y[static_cast<size_t>(m) * a.N + n] = __float2bfloat16_rn(v);
-                  }
-                }
+                const int m = m0 + j;
+                const float st = m < a.M ? __ldg(a.s_tok + m) : 0.f;
+                const float v = static_cast<float>(static_cast<int32_t>(r[j])) * st * sr;
+                const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+                asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_addr(dst)),
+                             "h"(*reinterpret_cast<const unsigned short*>(&hb))
+                             : "memory");
               } else {
-                int32_t* y = reinterpret_cast<int32_t*>(a.out);
-#pragma unroll
-                for (int j = 0; j < CW; ++j) {
-                  const int m = m0 + j;
-                  if (m < a.M) y[static_cast<size_t>(m) * a.N + n] = static_cast<int32_t>(r[j]) >> (W4 ? 4 : 0);
-                }
+                asm volatile("st.shared.b32 [%0], %1;" ::"r"(smem_addr(dst)),
+                             "r"(static_cast<uint32_t>(static_cast<int32_t>(r[j]) >> (W4 ? 4 : 0)))
+                             : "memory");
               }
             }
+            fence_proxy_async_smem();
+            if (et == 0) bulk_wait_group_read<0>();  // the previous chunk's half has been read
+            if (!epi_rendezvous()) {
+              staged_ok = false;
+              break;
+            }
+            if (et == 0) {
+              // rows past M and columns past N are clipped by the store
+              tma_store_2d(&tmY, xb, ta * GEMM_BM, m0);
+              bulk_commit_group();
+            }
+            sbuf ^= 1;
           }
+          if (!staged_ok) break;
         }
       }
       if (!seg.partial) {
@@ -603,7 +624,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
     }
     // the staged outputs must have been read before the CTA exits; the global
     // writes themselves complete before the grid does
-    if (!SWAP && lane == 0) bulk_wait_group_read<0>();
+    if (lane == 0) bulk_wait_group_read<0>();
   } else if (W4) {
     // ------------------------------------------------------------ int4 unpack
     const int ct = threadIdx.x - 192;  // 0..127
