@@ -87,6 +87,10 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::bar_offset(S));
   uint64_t* empty = full + GEMM_MAX_STAGES;
   uint64_t* conv = empty + GEMM_MAX_STAGES;
+  // int8: the second K atom of a stage lands on its own barrier, so the MMAs of
+  // the first atom start while the second is still in flight (the int4 kernel
+  // uses these barriers for its conversion hand-off instead)
+  uint64_t* full_hi = conv;
   uint64_t* tmem_full = conv + GEMM_MAX_STAGES;
   uint64_t* tmem_empty = tmem_full + 2;
   uint64_t* drain = tmem_empty + 2;
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&conv[s], 8);  // 4 converter warps in each CTA (leader's barrier)
+      mbar_init(&conv[s], W4 ? 8 : 1);  // int4: 4 converter warps in each CTA (leader's barrier)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
@@ -202,12 +206,18 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
                           brow, pol_b);
             }
           } else {
-            // both CTAs' tiles complete on the leader's barrier, which the leader arms
-            const uint32_t lead_full = mapa_shared(smem_addr(&full[s]), lead);
-            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (SM::A_BYTES + SM::B_BYTES));
+            // both CTAs' tiles complete on the leader's barriers, which the leader
+            // arms: atom 0 on full[s], atom 1 on full_hi[s]
+            static_assert(W4 || SM::KA == 2, "int8 pair stages hold two K atoms");
+            constexpr uint32_t ATOM_TX = 2u * (SM::A_ATOM + SM::B_ATOM);
+            if (rank == 0) {
+              mbar_arrive_expect_tx(&full[s], ATOM_TX);
+              mbar_arrive_expect_tx(&full_hi[s], ATOM_TX);
+            }
 #pragma unroll
             for (int j = 0; j < SM::KA; ++j) {
               // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
+              const uint32_t lead_full = mapa_shared(smem_addr(j == 0 ? &full[s] : &full_hi[s]), lead);
               const int k0 = (kb * SM::KA + j) * GEMM_BK;
               tma_load_2d_pair(st + j * SM::A_ATOM, &tmA, lead_full, k0, arow, pol_a);
               tma_load_2d_pair(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, lead_full, k0, brow, pol_b);
@@ -253,6 +263,13 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
           const uint32_t sb = sa + SM::A_BYTES;
 #pragma unroll
           for (int j = 0; j < SM::KA; ++j) {
+            if (!W4 && j == 1) {
+              if (!mbar_wait(&full_hi[s], ph, abort_flag, SITE_MMA_FULL)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
 #pragma unroll
             for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
               mma_s8_pair(d, sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K),
@@ -260,6 +277,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
                           (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u);
             }
           }
+          if (!ok) break;
           mma_commit_pair_mc(&empty[s], pair_mask);
         }
         if (!ok) break;
@@ -428,14 +446,13 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
               const int c0 = oc * (OC / 32);
 #pragma unroll
               for (int j4 = 0; j4 < 8; ++j4) {
-                const uint4 p0 = *reinterpret_cast<const uint4*>(rb + (c0 * 8 + j4) * 512 + lane * 16);
+                const uint4 p0 = ld_shared_v4(rb + (c0 * 8 + j4) * 512 + lane * 16);
                 r0[4 * j4] += p0.x;
                 r0[4 * j4 + 1] += p0.y;
                 r0[4 * j4 + 2] += p0.z;
                 r0[4 * j4 + 3] += p0.w;
                 if (OC == 64) {
-                  const uint4 p1 =
-                      *reinterpret_cast<const uint4*>(rb + ((c0 + 1) * 8 + j4) * 512 + lane * 16);
+                  const uint4 p1 = ld_shared_v4(rb + ((c0 + 1) * 8 + j4) * 512 + lane * 16);
                   r1[4 * j4] += p1.x;
                   r1[4 * j4 + 1] += p1.y;
                   r1[4 * j4 + 2] += p1.z;

@@ -760,11 +760,13 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
         if (need) sumsq = s64;
       }
     }
-    double rowfac = ROT ? 1.0 / 16.0 : 1.0;
-    if (NORM) rowfac *= 1.0 / sqrt(sumsq / static_cast<double>(a.K) + static_cast<double>(a.eps));
     const float inv = amax > 0.f ? 127.0f / amax : 0.0f;
-    if (row_ok && t == 0)
+    if (row_ok && t == 0) {
+      // the per-row scale is needed by one thread only
+      double rowfac = ROT ? 1.0 / 16.0 : 1.0;
+      if (NORM) rowfac *= 1.0 / sqrt(sumsq / static_cast<double>(a.K) + static_cast<double>(a.eps));
       a.s_tok[row] = amax > 0.f ? static_cast<float>(static_cast<double>(amax) * rowfac / 127.0) : 0.0f;
+    }
     act3_store<ROT>(a.xq + static_cast<size_t>(row_ok ? row : 0) * a.K, a.K, g, L, row_ok && g < G,
                     v, inv);
   }
