@@ -24,6 +24,11 @@ Everything is plain numpy in float64, written from the model cards' prose:
 * "Qwen3-VL 8B - INT8 ConvRot", "Layer and group selection": an input width
   that the group size does not divide falls back to plain row-wise INT8
   (``group = 0`` here).
+* "Qwen3-VL-8B-Heretic-1.3.0 - INT8 ConvRot (ComfyUI)", "Precision layout":
+  the quantised projections include mlp.gate_proj, mlp.up_proj and
+  mlp.down_proj; the MOSS-Image card's "How it was made" folds down_proj's
+  SmoothQuant scales into up_proj's rows.  The pages do not name the MLP's
+  activation; the Qwen-family reading down(SiLU(gate(x)) * up(x)) is taken.
 * "MossInt4", "Format": the convrot_w4a4 layout - 256-wide Hadamard, signed
   4-bit codes two per byte, one F32 scale per row chosen by a per-row clip
   search; activations stay 8-bit.
@@ -35,7 +40,10 @@ int4) and round-half-even; a zero row gets scale 0 and all-zero codes; the
 RMSNorm is x * (mean(x^2) + eps)^-1/2 * (1 + w) with no intermediate rounding;
 the int4 clip grid is clip_lo + (clip_hi - clip_lo) * i / (steps - 1), error
 is the row's sum of squared reconstruction errors, ties keep the smaller clip;
-the low nibble of byte j holds code 2j.
+the low nibble of byte j holds code 2j; gate and up rows of the fused MLP
+linear alternate in blocks of 16 rows, g and u are not rounded before
+SiLU(g) * u, and only h is rounded to bf16; the down_proj fold into up_proj's
+rows is applied to their row scales (exact for per-row quantisation).
 
 Parity status: every function below is pinned by ``tests/test_oracle.py``
 (closed forms, invariants, brute force on tiny inputs, library routines for
@@ -297,6 +305,22 @@ def linear_forward(x, Wq, s_row, group: int = GROUP, norm_w=None, eps: float = 1
 # --------------------------------------------------------------------------
 # SmoothQuant calibration used to prepare the synthetic norm-carrying layer
 # --------------------------------------------------------------------------
+def smoothquant_scales_of(a, W, alpha: float = 0.5, s_min: float = 1e-5, s_max: float = 1e5):
+    """Per input channel s_c = max_m|a[m,c]|^alpha / max_n|W[n,c]|^(1-alpha).
+
+    ``a`` [M, K] is the activation exactly as it reaches the linear (MOSS-Image
+    card, "How it was made": SmoothQuant, alpha 0.5, per input channel).  s is
+    clamped to [s_min, s_max]; a channel whose activation or weight column is
+    all zero keeps s = 1.
+    """
+    ax = np.max(np.abs(np.asarray(a, dtype=np.float64)), axis=0)
+    aw = np.max(np.abs(np.asarray(W, dtype=np.float64)), axis=0)
+    ok = (ax > 0) & (aw > 0)
+    s = np.where(ok, np.power(np.where(ok, ax, 1.0), alpha)
+                 / np.power(np.where(ok, aw, 1.0), 1.0 - alpha), 1.0)
+    return np.clip(s, s_min, s_max)
+
+
 def smoothquant_scales(x, norm_w, eps: float, W, alpha: float = 0.5,
                        s_min: float = 1e-5, s_max: float = 1e5):
     """Per input channel s_c = max_m|a[m,c]|^alpha / max_n|W[n,c]|^(1-alpha).
@@ -308,12 +332,77 @@ def smoothquant_scales(x, norm_w, eps: float, W, alpha: float = 0.5,
     (s, w_folded) with w_folded = (1 + w) / s - 1, the stored norm weight;
     the weight is then used as W * diag(s).
     """
-    a = rmsnorm(x, norm_w, eps)
-    ax = np.max(np.abs(a), axis=0)
-    aw = np.max(np.abs(np.asarray(W, dtype=np.float64)), axis=0)
-    ok = (ax > 0) & (aw > 0)
-    s = np.where(ok, np.power(np.where(ok, ax, 1.0), alpha)
-                 / np.power(np.where(ok, aw, 1.0), 1.0 - alpha), 1.0)
-    s = np.clip(s, s_min, s_max)
+    s = smoothquant_scales_of(rmsnorm(x, norm_w, eps), W, alpha, s_min, s_max)
     w_folded = (1.0 + np.asarray(norm_w, dtype=np.float64)) / s - 1.0
     return s, w_folded
+
+
+# --------------------------------------------------------------------------
+# MLP boundary: gate/up linear with SiLU(gate) * up, and the down_proj fold
+# --------------------------------------------------------------------------
+SWIGLU_BLOCK = 16  # gate and up rows alternate in blocks of this many rows
+
+
+def silu(z) -> np.ndarray:
+    """SiLU(z) = z * sigmoid(z) = z / (1 + exp(-z)), float64.
+
+    Evaluated as z * e / (1 + e) with e = exp(z) for z < 0 so that exp never
+    overflows; both forms are the same function.
+    """
+    z = np.asarray(z, dtype=np.float64)
+    pos = z >= 0
+    ez = np.exp(np.where(pos, -z, z))          # in (0, 1]
+    sig = np.where(pos, 1.0 / (1.0 + ez), ez / (1.0 + ez))
+    return z * sig
+
+
+def interleave_gate_up(Wg, Wu, block: int = SWIGLU_BLOCK) -> np.ndarray:
+    """Rows of gate and up in alternating blocks: [g0..g15, u0..u15, g16..].
+
+    Wg, Wu [I, ...] -> [2I, ...]; row r of the result is gate row
+    block*(r // (2 block)) + r % (2 block) when r % (2 block) < block, else
+    the up row with the same index.  I % block == 0.  One tile row of 2*block
+    accumulators then holds matching gate and up columns, which lets the
+    GEMM epilogue form SiLU(gate) * up without another pass.
+    """
+    Wg = np.asarray(Wg)
+    Wu = np.asarray(Wu)
+    if Wg.shape != Wu.shape or Wg.shape[0] % block:
+        raise ValueError("gate and up must have the same shape with rows a multiple of the block")
+    I = Wg.shape[0]
+    out = np.empty((2 * I,) + Wg.shape[1:], dtype=np.result_type(Wg, Wu))
+    gv = Wg.reshape((I // block, block) + Wg.shape[1:])
+    uv = Wu.reshape((I // block, block) + Wu.shape[1:])
+    ov = out.reshape((I // block, 2, block) + Wg.shape[1:])
+    ov[:, 0] = gv
+    ov[:, 1] = uv
+    return out
+
+
+def swiglu_linear(Xq, s_tok, Wq_gu, s_row_gu, block: int = SWIGLU_BLOCK):
+    """h = SiLU(g) * u from one W8A8 GEMM over interleaved gate/up weights.
+
+    g and u are the dequantised products acc * s_tok * s_row (float64, no
+    rounding before the activation); h [M, I] is rounded once to bf16.  This
+    is the down_proj input of a Qwen MLP block, down(SiLU(gate(x)) * up(x)).
+    Returns (h_bf16, h64, y64) with y64 the interleaved [M, 2I] products.
+    """
+    acc = int_matmul(Xq, Wq_gu)
+    y = dequant(acc, s_tok, s_row_gu)
+    M, N2 = y.shape
+    yv = y.reshape(M, N2 // (2 * block), 2, block)
+    g = yv[:, :, 0, :].reshape(M, N2 // 2)
+    u = yv[:, :, 1, :].reshape(M, N2 // 2)
+    h = silu(g) * u
+    return to_bf16(h), h, y
+
+
+def fold_smooth_into_rows(s_row, smooth) -> np.ndarray:
+    """Fold a per-channel scale 1/s into the rows of a row-quantised weight.
+
+    down_proj's SmoothQuant scale goes "into up_proj's rows" (MOSS-Image card,
+    "How it was made").  Each row of a ConvRot weight is rotated and quantised
+    on its own with an absmax scale, so dividing row c by s_c leaves its codes
+    unchanged and divides its scale: the fold is s_row[c] / s_c.
+    """
+    return np.asarray(s_row, dtype=np.float64) / np.asarray(smooth, dtype=np.float64)

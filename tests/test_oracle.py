@@ -366,3 +366,102 @@ def test_zero_row_with_zero_eps_stays_zero():
     q, s, v = ref.rotate_quant_act(x, norm_w=np.zeros(256), eps=0.0)
     assert s[0] == 0.0 and not q[0].any() and np.isfinite(v).all()
     assert s[1] > 0
+
+
+# ---------------------------------------------------------------- MLP boundary
+def test_silu_matches_library_logistic():
+    from scipy.special import expit
+    rng = np.random.default_rng(21)
+    z = np.concatenate([rng.uniform(-40, 40, 4000), [0.0, 1e-300, -1e-300, 700.0, -700.0, -1e4]])
+    want = z * expit(z)
+    got = ref.silu(z)
+    assert np.all(np.isfinite(got))
+    assert np.max(np.abs(got - want) / np.maximum(np.abs(want), 1e-300)) < 1e-14
+    assert ref.silu(np.array([0.0]))[0] == 0.0
+
+
+def test_silu_odd_part_identity():
+    # silu(z) - silu(-z) = z * (sigmoid(z) + sigmoid(-z)) = z for every z
+    z = np.linspace(-30, 30, 2001)
+    assert np.max(np.abs(ref.silu(z) - ref.silu(-z) - z)) < 1e-13
+    # and the even part is z * tanh(z / 2) / ... : silu(z) + silu(-z) = z tanh(z/2)
+    assert np.max(np.abs(ref.silu(z) + ref.silu(-z) - z * np.tanh(z / 2))) < 1e-12
+
+
+def test_interleave_gate_up_brute_force():
+    I, K, B = 48, 3, ref.SWIGLU_BLOCK
+    Wg = np.arange(I * K).reshape(I, K)
+    Wu = 1000 + np.arange(I * K).reshape(I, K)
+    out = ref.interleave_gate_up(Wg, Wu)
+    assert out.shape == (2 * I, K)
+    for r in range(2 * I):
+        blk, w = divmod(r, 2 * B)
+        src = Wg if w < B else Wu
+        assert np.array_equal(out[r], src[blk * B + (w % B)])
+    # every source row appears exactly once
+    seen = sorted(map(tuple, out.tolist()))
+    assert seen == sorted(map(tuple, np.concatenate([Wg, Wu]).tolist()))
+    with pytest.raises(ValueError):
+        ref.interleave_gate_up(Wg[:40], Wu[:40])
+
+
+def test_swiglu_linear_is_silu_of_gate_times_up():
+    rng = np.random.default_rng(22)
+    M, I, K = 5, 32, 64
+    Xq = rng.integers(-127, 128, (M, K))
+    Wg = rng.integers(-127, 128, (I, K))
+    Wu = rng.integers(-127, 128, (I, K))
+    s_tok = rng.uniform(1e-4, 1e-3, M)
+    sg = rng.uniform(1e-4, 1e-3, I)
+    su = rng.uniform(1e-4, 1e-3, I)
+    hb, h, _ = ref.swiglu_linear(Xq, s_tok, ref.interleave_gate_up(Wg, Wu),
+                                 ref.interleave_gate_up(sg, su))
+    _, yg, _ = ref.int8_linear(Xq, s_tok, Wg, sg)
+    _, yu, _ = ref.int8_linear(Xq, s_tok, Wu, su)
+    np.testing.assert_array_equal(h, ref.silu(yg) * yu)
+    np.testing.assert_array_equal(hb, ref.to_bf16(ref.silu(yg) * yu))
+    # a zero up scale or a zero gate row gives exactly zero
+    hb0, _, _ = ref.swiglu_linear(Xq, s_tok, ref.interleave_gate_up(Wg, Wu),
+                                  ref.interleave_gate_up(sg, np.zeros(I)))
+    assert not np.any(hb0)
+    hb1, _, _ = ref.swiglu_linear(Xq, s_tok, ref.interleave_gate_up(np.zeros_like(Wg), Wu),
+                                  ref.interleave_gate_up(sg, su))
+    assert not np.any(hb1)
+
+
+def test_smoothquant_scales_of_closed_form():
+    a = np.array([[2.0, -8.0, 0.0], [1.0, 4.0, 0.0]])
+    W = np.array([[0.5, 1.0, 3.0], [-2.0, 0.25, 1.0]])
+    s = ref.smoothquant_scales_of(a, W, alpha=0.5)
+    assert s[0] == pytest.approx(math.sqrt(2.0) / math.sqrt(2.0), rel=1e-15)
+    assert s[1] == pytest.approx(math.sqrt(8.0) / math.sqrt(1.0), rel=1e-15)
+    assert s[2] == 1.0                          # all-zero activation column
+    # alpha = 1 moves everything into the weight: s = max |a|
+    np.testing.assert_allclose(ref.smoothquant_scales_of(a, W, alpha=1.0)[:2], [2.0, 8.0], rtol=1e-15)
+    # scaling one activation column by t scales its s by t^alpha
+    a2 = a.copy()
+    a2[:, 1] *= 9.0
+    assert ref.smoothquant_scales_of(a2, W)[1] == pytest.approx(3.0 * s[1], rel=1e-14)
+
+
+def test_down_proj_fold_into_up_rows_preserves_the_mlp():
+    rng = np.random.default_rng(23)
+    M, H, I = 8, 256, 256
+    x = rng.standard_normal((M, H))
+    Wg = rng.standard_normal((I, H)) * 0.05
+    Wu = rng.standard_normal((I, H)) * 0.05
+    Wd = rng.standard_normal((H, I)) * 0.05
+    h = ref.silu(x @ Wg.T) * (x @ Wu.T)
+    h[:, 7] *= 100.0                                 # an outlier channel of the down input
+    s = ref.smoothquant_scales_of(h, Wd)
+    assert np.argmax(s) == 7
+    # (h / s) (Wd diag(s))^T == h Wd^T
+    lhs = (h / s[None, :]) @ (Wd * s[None, :]).T
+    rhs = h @ Wd.T
+    assert np.max(np.abs(lhs - rhs)) < 1e-12 * np.max(np.abs(rhs)) * 100
+    # dividing up's rows by s before quantisation leaves the codes and divides
+    # the row scales: the fold can be applied to s_row
+    q0, s0, _ = ref.quantize_weight(Wu)
+    q1, s1, _ = ref.quantize_weight(Wu / s[:, None])
+    np.testing.assert_array_equal(q0, q1)
+    np.testing.assert_allclose(ref.fold_smooth_into_rows(s0, s), s1, rtol=2e-7)
