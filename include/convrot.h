@@ -150,6 +150,10 @@ convrot_status convrot_quantize_weight_w4(const void* W, int N, int K, int group
  * x bf16 [M, K], norm_w fp32 [K], W bf16 [N, K] in; smooth, norm_w_folded
  * fp32 [K] out; norm_w_folded must not alias norm_w (both outputs are
  * used as scratch for the column maxima before the final values are written).
+ * norm_w may be NULL for a linear without a preceding norm (down_proj, whose
+ * input is the MLP's SiLU(gate) * up): then a = x, the scales are folded into
+ * the rows that produce x instead (convrot_fold_row_scales), and
+ * norm_w_folded is scratch only (its contents on return are unspecified).
  * K % 16 == 0.
  */
 convrot_status convrot_smoothquant_calibrate(const void* x, int M, int K, const float* norm_w,
@@ -214,6 +218,53 @@ convrot_status convrot_w4a8_linear(const int8_t* Xq, const float* s_tok, const u
                                    const float* s_row, int M, int N, int K, void* Y,
                                    void* workspace, size_t workspace_bytes,
                                    convrot_stream_t stream);
+
+/*
+ * MLP boundary: the gate/up projections of an MLP block as one W8A8 GEMM
+ * whose epilogue forms the down_proj input (the Heretic card's "Precision
+ * layout" quantises mlp.gate_proj, mlp.up_proj and mlp.down_proj; the block
+ * computes down(SiLU(gate(x)) * up(x))).
+ *   Wq_gu int8 [2I, K]: gate and up rows interleaved in blocks of 16 (see
+ *         convrot_interleave_gate_up), s_row_gu fp32 [2I] likewise;
+ *   g[m,i], u[m,i] = float(acc) * s_tok[m] * s_row   of the matching rows;
+ *   H[m,i] = bf16_rn(SiLU(g) * u),  SiLU(g) = g / (1 + exp(-g))   (fp32).
+ * Xq int8 [M, K], s_tok fp32 [M] in; H bf16 [M, I] out (16-byte aligned).
+ * I % 16 == 0; K as convrot_int8_linear.  H then goes through
+ * convrot_rotate_quant_act (no norm) into the down_proj linear.
+ * workspace: at least convrot_swiglu_workspace_bytes(M, I, K, bits) bytes,
+ * with the rules of convrot_int8_linear.
+ */
+size_t convrot_swiglu_workspace_bytes(int M, int I, int K, int weight_bits);
+convrot_status convrot_int8_linear_swiglu(const int8_t* Xq, const float* s_tok,
+                                          const int8_t* Wq_gu, const float* s_row_gu, int M,
+                                          int I, int K, void* H, void* workspace,
+                                          size_t workspace_bytes, convrot_stream_t stream);
+/* The same on int4 weights (Wq4_gu uint8 [2I, K/2], layout of convrot_w4a8_linear). */
+convrot_status convrot_w4a8_linear_swiglu(const int8_t* Xq, const float* s_tok,
+                                          const uint8_t* Wq4_gu, const float* s_row_gu, int M,
+                                          int I, int K, void* H, void* workspace,
+                                          size_t workspace_bytes, convrot_stream_t stream);
+
+/*
+ * Offline layout for convrot_*_linear_swiglu: out row r is gate row
+ * 16 (r / 32) + r % 32 when r % 32 < 16, else up row 16 (r / 32) + r % 32 - 16.
+ * Wg, Wu [I rows of row_bytes] in, out [2I rows] out; works on bf16 weights,
+ * quantised rows (int8 or packed int4) and the fp32 row scales alike.
+ * I % 16 == 0, row_bytes % 4 == 0, pointers 4-byte aligned; out must not
+ * overlap the inputs.
+ */
+convrot_status convrot_interleave_gate_up(const void* Wg, const void* Wu, int I,
+                                          size_t row_bytes, void* out, convrot_stream_t stream);
+
+/*
+ * Folds a per-channel SmoothQuant scale into the rows of a row-quantised
+ * weight: s_row[i] /= smooth[i], in place, fp32.  Used for down_proj, whose
+ * scales go "into up_proj's rows" (MOSS-Image card, "How it was made"): each
+ * ConvRot row is rotated and quantised on its own with an absmax scale, so
+ * dividing row i by smooth[i] leaves its codes and divides its scale.
+ */
+convrot_status convrot_fold_row_scales(float* s_row, const float* smooth, int n,
+                                       convrot_stream_t stream);
 
 /*
  * Allocation-free W8A8 linear.  The model cards have no counterpart: this is

@@ -20,7 +20,9 @@ __all__ = [
     "convrot_quantize_weight", "convrot_quantize_weight_w4", "convrot_smoothquant_calibrate",
     "convrot_rotate_quant_act", "convrot_linear_workspace_bytes", "convrot_int8_linear",
     "convrot_w4a8_linear", "convrot_int8_linear_noalloc", "convrot_int8_gemm_s32", "convrot_w4a8_gemm_s32",
-    "Workspace", "ConvRotLinear",
+    "convrot_swiglu_workspace_bytes", "convrot_int8_linear_swiglu", "convrot_w4a8_linear_swiglu",
+    "convrot_interleave_gate_up", "convrot_fold_row_scales",
+    "Workspace", "ConvRotLinear", "ConvRotMLP",
 ]
 
 
@@ -101,11 +103,14 @@ def convrot_quantize_weight_w4(W: torch.Tensor, group: int = 256,
     return Wq4, s_row
 
 
-def convrot_smoothquant_calibrate(x: torch.Tensor, norm_w: torch.Tensor, W: torch.Tensor,
+def convrot_smoothquant_calibrate(x: torch.Tensor, norm_w: Optional[torch.Tensor], W: torch.Tensor,
                                   eps: float = 1e-6, alpha: float = 0.5):
+    """SmoothQuant scales of the linear W fed by x (norm_w None: x reaches W as
+    it is, and the second result is scratch)."""
     _need(x, torch.bfloat16, "x", 2)
     _need(W, torch.bfloat16, "W", 2)
-    _need(norm_w, torch.float32, "norm_w", 1)
+    if norm_w is not None:
+        _need(norm_w, torch.float32, "norm_w", 1)
     M, K = x.shape
     N = W.shape[0]
     smooth = torch.empty(K, dtype=torch.float32, device=x.device)
@@ -238,6 +243,62 @@ def convrot_w4a8_gemm_s32(Xq, Wq4, workspace: Optional[Workspace] = None):
     return acc
 
 
+# ---------------------------------------------------------------- MLP boundary
+def convrot_swiglu_workspace_bytes(M: int, I: int, K: int, weight_bits: int = 8) -> int:
+    return int(lib().convrot_swiglu_workspace_bytes(M, I, K, weight_bits))
+
+
+def _swiglu(fn, Xq, s_tok, Wq_gu, s_row_gu, w4, out, workspace):
+    M, N2, K = _gemm_check(Xq, Wq_gu, w4)
+    _need(s_tok, torch.float32, "s_tok", 1)
+    _need(s_row_gu, torch.float32, "s_row_gu", 1)
+    if N2 % 2:
+        raise ValueError("the gate/up weight must have an even number of rows")
+    I = N2 // 2
+    H = torch.empty(M, I, dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    ws, wn = _workspace(Xq.device, convrot_swiglu_workspace_bytes(M, I, K, 4 if w4 else 8), workspace)
+    _check(fn, getattr(lib(), fn)(
+        _ptr(Xq), _ptr(s_tok), _ptr(Wq_gu), _ptr(s_row_gu), M, I, K, _ptr(H), ws, wn,
+        _stream(Xq.device)))
+    return H
+
+
+def convrot_int8_linear_swiglu(Xq, s_tok, Wq_gu, s_row_gu, out=None,
+                               workspace: Optional[Workspace] = None):
+    """H = bf16(SiLU(gate) * up) from interleaved gate/up rows (I = rows / 2)."""
+    return _swiglu("convrot_int8_linear_swiglu", Xq, s_tok, Wq_gu, s_row_gu, False, out, workspace)
+
+
+def convrot_w4a8_linear_swiglu(Xq, s_tok, Wq4_gu, s_row_gu, out=None,
+                               workspace: Optional[Workspace] = None):
+    return _swiglu("convrot_w4a8_linear_swiglu", Xq, s_tok, Wq4_gu, s_row_gu, True, out, workspace)
+
+
+def convrot_interleave_gate_up(Wg: torch.Tensor, Wu: torch.Tensor) -> torch.Tensor:
+    """Rows of gate and up in alternating blocks of 16 (any dtype, 1-D or 2-D)."""
+    if Wg.shape != Wu.shape or Wg.dtype != Wu.dtype or Wg.device != Wu.device:
+        raise ValueError("gate and up must match in shape, dtype and device")
+    if not (Wg.is_cuda and Wg.is_contiguous() and Wu.is_contiguous()):
+        raise ValueError("gate and up must be contiguous CUDA tensors")
+    I = Wg.shape[0]
+    row_bytes = Wg.numel() // max(I, 1) * Wg.element_size()
+    out = torch.empty((2 * I,) + tuple(Wg.shape[1:]), dtype=Wg.dtype, device=Wg.device)
+    _check("convrot_interleave_gate_up", lib().convrot_interleave_gate_up(
+        _ptr(Wg), _ptr(Wu), I, row_bytes, _ptr(out), _stream(Wg.device)))
+    return out
+
+
+def convrot_fold_row_scales(s_row: torch.Tensor, smooth: torch.Tensor) -> torch.Tensor:
+    """s_row /= smooth in place (a SmoothQuant scale folded into weight rows)."""
+    _need(s_row, torch.float32, "s_row", 1)
+    _need(smooth, torch.float32, "smooth", 1)
+    if s_row.shape != smooth.shape:
+        raise ValueError("s_row and smooth must have the same length")
+    _check("convrot_fold_row_scales", lib().convrot_fold_row_scales(
+        _ptr(s_row), _ptr(smooth), s_row.numel(), _stream(s_row.device)))
+    return s_row
+
+
 class ConvRotLinear:
     """A quantised linear layer: prepared weights plus the per-token forward.
 
@@ -271,5 +332,48 @@ class ConvRotLinear:
         if self.weight_bits == 8:
             return convrot_int8_linear(Xq, s_tok, self.Wq, self.s_row, out, self.workspace)
         return convrot_w4a8_linear(Xq, s_tok, self.Wq, self.s_row, out, self.workspace)
+
+    __call__ = forward
+
+
+class ConvRotMLP:
+    """The MLP block down(SiLU(gate(x)) * up(x)) of the quantised decoder layer.
+
+    forward(x) = rotate-quantise (with the fused RMSNorm) -> one gate/up GEMM
+    whose epilogue writes H = SiLU(g) * u -> rotate-quantise H -> down_proj.
+    With calibration input, SmoothQuant scales are folded into the norm
+    weight (gate/up input) and into up_proj's row scales (down_proj input),
+    as the MOSS-Image card's "How it was made" describes.
+    """
+
+    def __init__(self, Wg: torch.Tensor, Wu: torch.Tensor, Wd: torch.Tensor, *,
+                 norm_w: Optional[torch.Tensor] = None, x_calib: Optional[torch.Tensor] = None,
+                 group: int = 256, eps: float = 1e-6, alpha: float = 0.5):
+        self.group, self.eps = group, eps
+        self.I, self.H = Wg.shape
+        self.workspace = Workspace(Wg.device.index)
+        col = None
+        self.norm_w = norm_w
+        if x_calib is not None and norm_w is not None:
+            col, self.norm_w = convrot_smoothquant_calibrate(x_calib, norm_w, torch.cat([Wg, Wu]), eps, alpha)
+        Wq_g, s_g = convrot_quantize_weight(Wg, group, col)
+        Wq_u, s_u = convrot_quantize_weight(Wu, group, col)
+        self.Wq_gu = convrot_interleave_gate_up(Wq_g, Wq_u)
+        s_gu = convrot_interleave_gate_up(s_g, s_u)
+        smooth_d = None
+        if x_calib is not None:
+            Xq, s_tok = convrot_rotate_quant_act(x_calib, group, self.norm_w, eps)
+            h = convrot_int8_linear_swiglu(Xq, s_tok, self.Wq_gu, s_gu, workspace=self.workspace)
+            smooth_d, _ = convrot_smoothquant_calibrate(h, None, Wd, eps, alpha)
+            convrot_fold_row_scales(s_u, smooth_d)
+            s_gu = convrot_interleave_gate_up(s_g, s_u)
+        self.s_gu = s_gu
+        self.Wq_d, self.s_d = convrot_quantize_weight(Wd, group, smooth_d)
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        Xq, s_tok = convrot_rotate_quant_act(x, self.group, self.norm_w, self.eps)
+        h = convrot_int8_linear_swiglu(Xq, s_tok, self.Wq_gu, self.s_gu, workspace=self.workspace)
+        Hq, s_h = convrot_rotate_quant_act(h, self.group, None, self.eps)
+        return convrot_int8_linear(Hq, s_h, self.Wq_d, self.s_d, out, self.workspace)
 
     __call__ = forward

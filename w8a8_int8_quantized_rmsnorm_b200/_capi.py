@@ -49,6 +49,13 @@ SIGNATURES = {
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "convrot_w4a8_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                                     c_void_p, c_void_p, c_size_t, c_void_p]),
+    "convrot_swiglu_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "convrot_int8_linear_swiglu": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                                           c_void_p, c_void_p, c_size_t, c_void_p]),
+    "convrot_w4a8_linear_swiglu": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                                           c_void_p, c_void_p, c_size_t, c_void_p]),
+    "convrot_interleave_gate_up": (c_int, [c_void_p, c_void_p, c_int, c_size_t, c_void_p, c_void_p]),
+    "convrot_fold_row_scales": (c_int, [c_void_p, c_void_p, c_int, c_void_p]),
     "convrot_int8_linear_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                             c_int, c_void_p, c_void_p]),
     "convrot_int8_gemm_s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,

@@ -424,15 +424,25 @@ int split_units(int device) {
   return clusters;
 }
 
-int split_units_for(bool w4, bool s32, int device) {
-  if (w4) return 0;
-  const int c = s32 ? split_units<EPI_S32>(device) : split_units<EPI_BF16>(device);
+// `epi` is the epilogue mode (EPI_BF16, EPI_S32 or EPI_SWIGLU).
+int split_units_for(bool w4, int epi, int device) {
+  if (w4 || epi == EPI_SWIGLU) return 0;  // the split-K cluster mode is int8 and plain only
+  const int c = epi == EPI_S32 ? split_units<EPI_S32>(device) : split_units<EPI_BF16>(device);
   return c > 0 ? c : 0;
 }
 
-int pair_units_for(bool w4, bool s32, int device) {
-  if (w4) return s32 ? pair_units<true, EPI_S32>(device) : pair_units<true, EPI_BF16>(device);
-  return s32 ? pair_units<false, EPI_S32>(device) : pair_units<false, EPI_BF16>(device);
+int pair_units_for(bool w4, int epi, int device) {
+  if (w4) {
+    if (epi == EPI_SWIGLU) return pair_units<true, EPI_SWIGLU>(device);
+    return epi == EPI_S32 ? pair_units<true, EPI_S32>(device) : pair_units<true, EPI_BF16>(device);
+  }
+  if (epi == EPI_SWIGLU) return pair_units<false, EPI_SWIGLU>(device);
+  return epi == EPI_S32 ? pair_units<false, EPI_S32>(device) : pair_units<false, EPI_BF16>(device);
+}
+
+GemmPlan plan_for(int M, int N, int K, bool w4, int epi, const DeviceInfo& d) {
+  return plan_gemm(M, N, K, d.sms, pair_units_for(w4, epi, d.device), w4,
+                   split_units_for(w4, epi, d.device));
 }
 
 // `units` counts CTA pairs, or (SPLIT) clusters of two pairs.
@@ -495,13 +505,31 @@ convrot_status launch_gemm_bn(int bn, const CUtensorMap& ma, const CUtensorMap& 
   }
 }
 
+template <bool SWAP, bool W4>
+convrot_status launch_gemm_epi(int epi, int bn, const CUtensorMap& ma, const CUtensorMap& mb,
+                               const CUtensorMap& my, const GemmArgs& a, int grid, cudaStream_t st) {
+  if (epi == EPI_S32) return launch_gemm_bn<SWAP, W4, EPI_S32>(bn, ma, mb, my, a, grid, st);
+  if (epi == EPI_SWIGLU) return launch_gemm_bn<SWAP, W4, EPI_SWIGLU>(bn, ma, mb, my, a, grid, st);
+  return launch_gemm_bn<SWAP, W4, EPI_BF16>(bn, ma, mb, my, a, grid, st);
+}
+
+template <bool W4>
+convrot_status launch_pair_epi(int epi, const CUtensorMap& ma, const CUtensorMap& mb,
+                               const CUtensorMap& my, const GemmArgs& a, int units, cudaStream_t st) {
+  if (epi == EPI_S32) return launch_gemm_pair<W4, EPI_S32>(ma, mb, my, a, units, st);
+  if (epi == EPI_SWIGLU) return launch_gemm_pair<W4, EPI_SWIGLU>(ma, mb, my, a, units, st);
+  return launch_gemm_pair<W4, EPI_BF16>(ma, mb, my, a, units, st);
+}
+
+// epi = EPI_BF16 (Y bf16 [M, N]), EPI_S32 (acc int32 [M, N]) or EPI_SWIGLU
+// (H bf16 [M, N / 2] from interleaved gate/up weight rows).
 convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* s_tok,
-                        const float* s_row, int M, int N, int K, void* out, bool s32_out,
+                        const float* s_row, int M, int N, int K, void* out, int epi,
                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const GemmPlan p = plan_gemm(M, N, K, d.sms, pair_units_for(w4, s32_out, d.device), w4,
-                                split_units_for(w4, s32_out, d.device));
+  const bool s32_out = epi == EPI_S32;
+  const GemmPlan p = plan_for(M, N, K, w4, epi, d);
   const size_t need = ws_bytes(p);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CONVROT_ERR_WORKSPACE;
   if (need > 0 && !aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
@@ -522,15 +550,19 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
   // output map for the epilogues' TMA stores
   CUtensorMap my;
   std::memset(&my, 0, sizeof(my));
+  // the SwiGLU epilogue writes N / 2 columns: 64 per staged row, or 64 per
+  // 128-row tile of the swapped roles
+  const uint64_t out_cols = epi == EPI_SWIGLU ? N / 2 : N;
   if (!p.swap) {
     const bool ok = s32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_INT32, 32, 32, true)
-                            : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, 64, true);
+                            : make_map(&my, out, M, out_cols, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, 64, true);
     if (!ok) return CONVROT_ERR_CUDA;
   } else {
     // swapped roles: chunks of up to 32 tokens x 128 output columns, unswizzled
     const uint32_t cw = bn < 32 ? bn : 32;
+    const uint32_t box_cols = epi == EPI_SWIGLU ? 64 : 128;
     const bool ok = s32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_INT32, cw, 128, false)
-                            : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cw, 128, false);
+                            : make_map(&my, out, M, out_cols, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cw, box_cols, false);
     if (!ok) return CONVROT_ERR_CUDA;
   }
 
@@ -557,28 +589,17 @@ convrot_status run_gemm(const int8_t* Xq, const void* Wq, bool w4, const float* 
                   : nullptr;
   const CUtensorMap& ma = p.swap ? mw : mx;
   const CUtensorMap& mb = p.swap ? mx : mw;
-  if (p.split)
+  if (p.split)  // never for EPI_SWIGLU (split_units_for gives no clusters)
     return s32_out ? launch_gemm_pair<false, EPI_S32, true>(ma, mb, my, a, p.grid, st)
                    : launch_gemm_pair<false, EPI_BF16, true>(ma, mb, my, a, p.grid, st);
-  if (p.pair) {
-    if (w4)
-      return s32_out ? launch_gemm_pair<true, EPI_S32>(ma, mb, my, a, p.grid, st)
-                     : launch_gemm_pair<true, EPI_BF16>(ma, mb, my, a, p.grid, st);
-    return s32_out ? launch_gemm_pair<false, EPI_S32>(ma, mb, my, a, p.grid, st)
-                   : launch_gemm_pair<false, EPI_BF16>(ma, mb, my, a, p.grid, st);
-  }
-  if (w4) {
-    if (s32_out)
-      return p.swap ? launch_gemm_bn<true, true, EPI_S32>(bn, ma, mb, my, a, p.grid, st)
-                    : launch_gemm_bn<false, true, EPI_S32>(bn, ma, mb, my, a, p.grid, st);
-    return p.swap ? launch_gemm_bn<true, true, EPI_BF16>(bn, ma, mb, my, a, p.grid, st)
-                  : launch_gemm_bn<false, true, EPI_BF16>(bn, ma, mb, my, a, p.grid, st);
-  }
-  if (s32_out)
-    return p.swap ? launch_gemm_bn<true, false, EPI_S32>(bn, ma, mb, my, a, p.grid, st)
-                  : launch_gemm_bn<false, false, EPI_S32>(bn, ma, mb, my, a, p.grid, st);
-  return p.swap ? launch_gemm_bn<true, false, EPI_BF16>(bn, ma, mb, my, a, p.grid, st)
-                : launch_gemm_bn<false, false, EPI_BF16>(bn, ma, mb, my, a, p.grid, st);
+  if (p.pair)
+    return w4 ? launch_pair_epi<true>(epi, ma, mb, my, a, p.grid, st)
+              : launch_pair_epi<false>(epi, ma, mb, my, a, p.grid, st);
+  if (w4)
+    return p.swap ? launch_gemm_epi<true, true>(epi, bn, ma, mb, my, a, p.grid, st)
+                  : launch_gemm_epi<false, true>(epi, bn, ma, mb, my, a, p.grid, st);
+  return p.swap ? launch_gemm_epi<true, false>(epi, bn, ma, mb, my, a, p.grid, st)
+                : launch_gemm_epi<false, false>(epi, bn, ma, mb, my, a, p.grid, st);
 }
 
 convrot_status check_gemm_shape(int M, int N, int K, bool w4) {
@@ -730,8 +751,8 @@ convrot_status convrot_smoothquant_calibrate(const void* x, int M, int K, const 
                                              convrot_stream_t stream) {
   if (M <= 0 || N <= 0 || K <= 0 || K > CONVROT_MAX_K || K % 16) return CONVROT_ERR_SHAPE;
   if (!(alpha >= 0.f && alpha <= 1.f) || !(eps >= 0.f)) return CONVROT_ERR_SHAPE;
-  if (!x || !norm_w || !W || !smooth || !norm_w_folded) return CONVROT_ERR_NULL;
-  if (!aligned(x, 16) || !aligned(W, 16) || !aligned(norm_w, 4) || !aligned(smooth, 4) ||
+  if (!x || !W || !smooth || !norm_w_folded) return CONVROT_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(W, 16) || (norm_w && !aligned(norm_w, 4)) || !aligned(smooth, 4) ||
       !aligned(norm_w_folded, 4))
     return CONVROT_ERR_ALIGN;
   if (norm_w_folded == norm_w) return CONVROT_ERR_UNSUPPORTED;
@@ -754,8 +775,17 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return 0;
   // the bf16 and int32 outputs share the schedule, so either plan gives the size
-  return ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(weight_bits == 4, false, d.device), weight_bits == 4,
-                            split_units_for(weight_bits == 4, false, d.device)));
+  return ws_bytes(plan_for(M, N, K, weight_bits == 4, EPI_BF16, d));
+}
+
+size_t convrot_swiglu_workspace_bytes(int M, int I, int K, int weight_bits) {
+  if (I <= 0 || I % SWIGLU_BLOCK || I > (1 << 29)) return 0;
+  if (check_gemm_shape(M, 2 * I, K, weight_bits == 4) != CONVROT_OK) return 0;
+  if (weight_bits != 8 && weight_bits != 4) return 0;
+  if (M == 0) return 0;
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return 0;
+  return ws_bytes(plan_for(M, 2 * I, K, weight_bits == 4, EPI_SWIGLU, d));
 }
 
 static convrot_status linear_common(const int8_t* Xq, const float* s_tok, const void* Wq,
@@ -769,8 +799,67 @@ static convrot_status linear_common(const int8_t* Xq, const float* s_tok, const 
   if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(s_tok, 4) ||
       !aligned(s_row, 4))
     return CONVROT_ERR_ALIGN;
-  return run_gemm(Xq, Wq, w4, s_tok, s_row, M, N, K, Y, false, workspace, workspace_bytes,
+  return run_gemm(Xq, Wq, w4, s_tok, s_row, M, N, K, Y, EPI_BF16, workspace, workspace_bytes,
                   as_cuda(stream));
+}
+
+static convrot_status swiglu_common(const int8_t* Xq, const float* s_tok, const void* Wq_gu,
+                                    bool w4, const float* s_row_gu, int M, int I, int K, void* H,
+                                    void* workspace, size_t workspace_bytes,
+                                    convrot_stream_t stream) {
+  if (M < 0 || I <= 0 || I % SWIGLU_BLOCK || I > (1 << 29)) return CONVROT_ERR_SHAPE;
+  const convrot_status sh = check_gemm_shape(M, 2 * I, K, w4);
+  if (sh != CONVROT_OK) return sh;
+  if (M == 0) return CONVROT_OK;
+  if (!Xq || !s_tok || !Wq_gu || !s_row_gu || !H) return CONVROT_ERR_NULL;
+  if (!aligned(Xq, 16) || !aligned(Wq_gu, 16) || !aligned(H, 16) || !aligned(s_tok, 4) ||
+      !aligned(s_row_gu, 4))
+    return CONVROT_ERR_ALIGN;
+  return run_gemm(Xq, Wq_gu, w4, s_tok, s_row_gu, M, 2 * I, K, H, EPI_SWIGLU, workspace,
+                  workspace_bytes, as_cuda(stream));
+}
+
+convrot_status convrot_int8_linear_swiglu(const int8_t* Xq, const float* s_tok,
+                                          const int8_t* Wq_gu, const float* s_row_gu, int M,
+                                          int I, int K, void* H, void* workspace,
+                                          size_t workspace_bytes, convrot_stream_t stream) {
+  return swiglu_common(Xq, s_tok, Wq_gu, false, s_row_gu, M, I, K, H, workspace,
+                       workspace_bytes, stream);
+}
+
+convrot_status convrot_w4a8_linear_swiglu(const int8_t* Xq, const float* s_tok,
+                                          const uint8_t* Wq4_gu, const float* s_row_gu, int M,
+                                          int I, int K, void* H, void* workspace,
+                                          size_t workspace_bytes, convrot_stream_t stream) {
+  return swiglu_common(Xq, s_tok, Wq4_gu, true, s_row_gu, M, I, K, H, workspace,
+                       workspace_bytes, stream);
+}
+
+convrot_status convrot_interleave_gate_up(const void* Wg, const void* Wu, int I,
+                                          size_t row_bytes, void* out, convrot_stream_t stream) {
+  if (I <= 0 || I % SWIGLU_BLOCK || row_bytes == 0 || row_bytes % 4 ||
+      row_bytes > (static_cast<size_t>(1) << 30))
+    return CONVROT_ERR_SHAPE;
+  if (!Wg || !Wu || !out) return CONVROT_ERR_NULL;
+  if (!aligned(Wg, 4) || !aligned(Wu, 4) || !aligned(out, 4)) return CONVROT_ERR_ALIGN;
+  const size_t words = static_cast<size_t>(2) * I * (row_bytes / 4);
+  const int threads = 256;
+  const size_t want = (words + threads - 1) / threads;
+  const int blocks = static_cast<int>(std::min<size_t>(want, 148 * 16));
+  interleave_rows_kernel<<<blocks, threads, 0, as_cuda(stream)>>>(
+      static_cast<const uint32_t*>(Wg), static_cast<const uint32_t*>(Wu),
+      static_cast<uint32_t*>(out), static_cast<size_t>(I), row_bytes / 4);
+  return launch_status();
+}
+
+convrot_status convrot_fold_row_scales(float* s_row, const float* smooth, int n,
+                                       convrot_stream_t stream) {
+  if (n < 0) return CONVROT_ERR_SHAPE;
+  if (n == 0) return CONVROT_OK;
+  if (!s_row || !smooth) return CONVROT_ERR_NULL;
+  if (!aligned(s_row, 4) || !aligned(smooth, 4)) return CONVROT_ERR_ALIGN;
+  fold_row_scales_kernel<<<(n + 255) / 256, 256, 0, as_cuda(stream)>>>(s_row, smooth, n);
+  return launch_status();
 }
 
 convrot_status convrot_int8_linear(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
@@ -799,7 +888,7 @@ static convrot_status gemm_s32_common(const int8_t* Xq, const void* Wq, bool w4,
   if (M == 0 || N == 0) return CONVROT_OK;
   if (!Xq || !Wq || !acc) return CONVROT_ERR_NULL;
   if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(acc, 16)) return CONVROT_ERR_ALIGN;
-  return run_gemm(Xq, Wq, w4, nullptr, nullptr, M, N, K, acc, true, workspace, workspace_bytes,
+  return run_gemm(Xq, Wq, w4, nullptr, nullptr, M, N, K, acc, EPI_S32, workspace, workspace_bytes,
                   as_cuda(stream));
 }
 
@@ -871,8 +960,7 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
     return CONVROT_ERR_ALIGN;
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
-  const size_t need = ws_bytes(plan_gemm(M, N, K, d.sms, pair_units_for(false, false, d.device), false,
-                            split_units_for(false, false, d.device)));
+  const size_t need = ws_bytes(plan_for(M, N, K, false, EPI_BF16, d));
   if (need > kStaticWorkspaceBytes) return CONVROT_ERR_WORKSPACE;  // shape too large for the array
   void* ws = nullptr;
   if (need > 0) {
@@ -881,6 +969,6 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
     // the counters and accumulators this call uses must start at zero
     if (cudaMemsetAsync(ws, 0, need, as_cuda(stream)) != cudaSuccess) return CONVROT_ERR_CUDA;
   }
-  return run_gemm(Xq, Wq, false, s_tok, s_row, M, N, K, Y, false, ws,
+  return run_gemm(Xq, Wq, false, s_tok, s_row, M, N, K, Y, EPI_BF16, ws,
                   need > 0 ? kStaticWorkspaceBytes : 0, as_cuda(stream));
 }

@@ -63,6 +63,11 @@ __host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
 }
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
+// SiLU(gate) * up of the MLP boundary: the weight rows alternate in blocks of
+// SWIGLU_BLOCK gate rows and SWIGLU_BLOCK up rows, and the output has half as
+// many columns as the weight has rows
+constexpr int EPI_SWIGLU = 2;
+constexpr int SWIGLU_BLOCK = 16;
 
 // wait sites recorded in the device error word
 constexpr unsigned SITE_PROD_EMPTY = 1, SITE_MMA_FULL = 2, SITE_MMA_TMEM = 3, SITE_EPI_FULL = 4,
@@ -155,6 +160,27 @@ __device__ __forceinline__ void tile_coords(const GemmArgs& a, int tile, int& ta
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// SiLU(g) * u in fp32: g / (1 + e^-g) * u.  For g far below zero e^-g is
+// infinite and the quotient is a signed zero, the function's limit.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return g / (1.0f + __expf(-g)) * u;
+}
+
+// Sixteen outputs of the MLP boundary from one 32-column accumulator chunk
+// whose first 16 columns are gate rows and last 16 the matching up rows:
+// h_j = SiLU(acc_j * st * sr_j) * (acc_{16+j} * st * sr_{16+j}), as 8 bf16x2.
+__device__ __forceinline__ void swiglu16(const uint32_t (&r)[32], float st, const float (&sr)[32],
+                                         uint32_t (&w)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float g0 = static_cast<float>(static_cast<int32_t>(r[2 * j])) * st * sr[2 * j];
+    const float g1 = static_cast<float>(static_cast<int32_t>(r[2 * j + 1])) * st * sr[2 * j + 1];
+    const float u0 = static_cast<float>(static_cast<int32_t>(r[16 + 2 * j])) * st * sr[16 + 2 * j];
+    const float u1 = static_cast<float>(static_cast<int32_t>(r[17 + 2 * j])) * st * sr[17 + 2 * j];
+    w[j] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
+  }
 }
 
 // Shared-memory plan (offsets from a 1024-byte aligned base).
@@ -452,9 +478,57 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
           const int m = arow;
           const int m0 = ta * GEMM_BM + 32 * q;
           float st = 0.f;
-          if (EPI == EPI_BF16 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
+          if (EPI != EPI_S32 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
 #pragma unroll 1
-          for (int oc = 0; oc < BN / OC; ++oc) {
+          for (int oc = 0; oc < (EPI == EPI_SWIGLU ? BN / 128 : 0); ++oc) {
+            // MLP boundary: 128 accumulator columns (four blocks of 16 gate and
+            // 16 up columns) give the 64 outputs of one staged 128-byte row
+            uint8_t* buf = stage_buf + sbuf * 4096;
+            if (lane == 0) bulk_wait_group_read<1>();  // the store from two chunks ago has read buf
+            __syncwarp();
+            const int sw = lane & 7;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              const int cc = oc * 4 + c;  // 32-column chunk of the tile
+              uint32_t r[32];
+              if (!seg.partial) {
+                tmem_ld_32x32b_x32(tbase + cc * 32, r);
+                tmem_ld_wait();
+              } else {
+                // the tile's sum; leave the accumulator at zero for the next call
+                uint4* base = reinterpret_cast<uint4*>(acc_tile) + (cc * 4 + q) * 8 * 32 + lane;
+                uint4 v[8];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) v[j4] = __ldcg(base + j4 * 32);
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                  __stcg(base + j4 * 32, z);
+                  r[4 * j4] = v[j4].x;
+                  r[4 * j4 + 1] = v[j4].y;
+                  r[4 * j4 + 2] = v[j4].z;
+                  r[4 * j4 + 3] = v[j4].w;
+                }
+              }
+              const int n0 = tb * BN + cc * 32;
+              float sr[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sr[j] = n0 + j < a.N ? __ldg(a.s_row + n0 + j) : 0.f;
+              uint32_t w[8];
+              swiglu16(r, st, sr, w);
+              st_shared_v4(buf + lane * 128 + (((2 * c) ^ sw) << 4), w[0], w[1], w[2], w[3]);
+              st_shared_v4(buf + lane * 128 + (((2 * c + 1) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, buf, (tb * BN + oc * 128) / 2, m0);
+              bulk_commit_group();
+            }
+            sbuf ^= 1;
+          }
+#pragma unroll 1
+          for (int oc = 0; oc < (EPI == EPI_SWIGLU ? 0 : BN / OC); ++oc) {
             uint32_t r0[32], r1[32];
             if (!seg.partial) {
               tmem_ld_32x32b_x32(tbase + oc * OC, r0);
@@ -553,7 +627,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
           const int n = arow;
           const int nl = 32 * q + lane;  // column of this lane in the staged tile
           float sr = 0.f;
-          if (EPI == EPI_BF16 && n < a.N) sr = a.s_row[n] * (W4 ? 0.0625f : 1.0f);
+          if (EPI != EPI_S32 && n < a.N) sr = a.s_row[n] * (W4 ? 0.0625f : 1.0f);
           bool staged_ok = true;
 #pragma unroll 1
           for (int c = 0; c < BN / CW; ++c) {
@@ -582,8 +656,29 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
             }
             const int m0 = tb * BN + c * CW;
             uint8_t* xb = smem + SM::staging_offset(S) + sbuf * 16384;
+            if (EPI == EPI_SWIGLU) {
+              // MLP boundary, staged as [CW tokens][64 outputs]: each warp's
+              // lanes are one block, gate rows in lanes 0-15 and the matching
+              // up rows in lanes 16-31.  Of each token pair the low lanes form
+              // the even token's outputs and the high lanes the odd token's.
+              const bool upper = lane >= 16;
+              const int col = 16 * q + (lane & 15);
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
+              for (int j = 0; j < CW; j += 2) {
+                const float st0 = m0 + j < a.M ? __ldg(a.s_tok + m0 + j) : 0.f;
+                const float st1 = m0 + j + 1 < a.M ? __ldg(a.s_tok + m0 + j + 1) : 0.f;
+                const float v0 = static_cast<float>(static_cast<int32_t>(r[j])) * st0 * sr;
+                const float v1 = static_cast<float>(static_cast<int32_t>(r[j + 1])) * st1 * sr;
+                const float other = __shfl_xor_sync(0xffffffffu, upper ? v0 : v1, 16);
+                const float hv = upper ? silu_mul(other, v1) : silu_mul(v0, other);
+                const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+                asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_addr(xb + (j + (upper ? 1 : 0)) * 128 + col * 2)),
+                             "h"(*reinterpret_cast<const unsigned short*>(&hb))
+                             : "memory");
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < (EPI == EPI_SWIGLU ? 0 : CW); ++j) {
               uint8_t* dst = xb + j * (128 * ES) + nl * ES;
               if (EPI == EPI_BF16) {
                 const int m = m0 + j;
@@ -607,7 +702,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
             }
             if (et == 0) {
               // rows past M and columns past N are clipped by the store
-              tma_store_2d(&tmY, xb, ta * GEMM_BM, m0);
+              tma_store_2d(&tmY, xb, EPI == EPI_SWIGLU ? ta * GEMM_BM / 2 : ta * GEMM_BM, m0);
               bulk_commit_group();
             }
             sbuf ^= 1;

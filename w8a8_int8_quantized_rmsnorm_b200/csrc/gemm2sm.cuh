@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
                    const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
   using SM = Gemm2Smem<W4>;
   static_assert(!(SPLIT && W4), "the split-K cluster mode is int8 only");
+  static_assert(!(SPLIT && EPI == EPI_SWIGLU), "the split-K cluster mode has no SwiGLU epilogue");
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
   constexpr int BN = 256;
   constexpr uint32_t IDESC = idesc_s8s8s32(256, BN);
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
       float srl[FC / 32];
 #pragma unroll
       for (int c = 0; c < FC / 32; ++c) srl[c] = 0.f;
-      if (EPI == EPI_BF16) {
+      if (EPI != EPI_S32) {
         if (m < a.M) st = __ldg(a.s_tok + m) * (W4 ? 0.0625f : 1.0f);
 #pragma unroll
         for (int c = 0; c < FC / 32; ++c) {
@@ -432,7 +433,50 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
         finalize = *last_flag != 0;
         if (finalize) __threadfence();
       }
-      if (finalize) {
+      if (finalize && EPI == EPI_SWIGLU) {
+        // MLP boundary: the warp's 128 accumulator columns are four blocks of
+        // 16 gate and 16 up columns; their 64 outputs fill one staged 128-byte
+        // row per token, stored with one TMA store at column ncol0 / 2
+        if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read buf
+        __syncwarp();
+        const int sw = lane & 7;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // unrolled: srl[c] stays in registers
+          uint32_t r[32];
+          if (!seg.partial) {
+            tmem_ld_32x32b_x32(tq + fcol + 32 * c, r);
+            tmem_ld_wait();
+          } else {
+            // the tile's sum; leave the accumulator at zero for the next call
+            uint4* base = reinterpret_cast<uint4*>(acc_tile) + ((h * 4 + c) * 4 + q) * 8 * 32 + lane;
+            uint4 v[8];
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) v[j4] = __ldcg(base + j4 * 32);
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              __stcg(base + j4 * 32, z);
+              r[4 * j4] = v[j4].x;
+              r[4 * j4 + 1] = v[j4].y;
+              r[4 * j4 + 2] = v[j4].z;
+              r[4 * j4 + 3] = v[j4].w;
+            }
+          }
+          float sr[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sr[j] = __shfl_sync(0xffffffffu, srl[c], j);
+          uint32_t w[8];
+          swiglu16(r, st, sr, w);
+          st_shared_v4(buf + lane * 128 + (((2 * c) ^ sw) << 4), w[0], w[1], w[2], w[3]);
+          st_shared_v4(buf + lane * 128 + (((2 * c + 1) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmY, buf, ncol0 / 2, m0);
+          bulk_commit_group();
+        }
+      } else if (finalize) {
 #pragma unroll
         for (int oc = 0; oc < FC / OC; ++oc) {
           uint32_t r0[32], r1[32];

@@ -779,14 +779,17 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
 constexpr int CAL_ROWS = 64;
 
 // ax[c] = max over rows of |x[m,c] * r_m * (1 + w[c])|, as float bits in an
-// unsigned max (order-preserving for non-negative floats).
+// unsigned max (order-preserving for non-negative floats).  w == nullptr: the
+// activation reaches the linear as it is (ax[c] = max |x[m,c]|).
 __global__ void __launch_bounds__(256) calib_act_colmax(const uint16_t* x, int M, int K,
                                                         const float* w, float eps,
                                                         unsigned* axbits) {
   __shared__ float s_r[CAL_ROWS];
   const int m0 = blockIdx.x * CAL_ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int rr = warp; rr < CAL_ROWS; rr += 8) {
+  for (int rr = warp; rr < CAL_ROWS && w == nullptr; rr += 8)
+    if (lane == 0) s_r[rr] = 1.0f;
+  for (int rr = warp; rr < CAL_ROWS && w != nullptr; rr += 8) {
     const int m = m0 + rr;
     double acc = 0.0;
     if (m < M) {
@@ -801,7 +804,7 @@ __global__ void __launch_bounds__(256) calib_act_colmax(const uint16_t* x, int M
   }
   __syncthreads();
   for (int c = threadIdx.x; c < K; c += blockDim.x) {
-    const float mult = 1.0f + w[c];
+    const float mult = w != nullptr ? 1.0f + w[c] : 1.0f;
     float mx = 0.f;
     for (int rr = 0; rr < CAL_ROWS && m0 + rr < M; ++rr) {
       const float xv = __uint_as_float(static_cast<uint32_t>(x[static_cast<size_t>(m0 + rr) * K + c]) << 16);
@@ -834,7 +837,33 @@ __global__ void __launch_bounds__(256) calib_finalize(const float* w, int K, flo
   if (ax > 0.0 && aw > 0.0) s = pow(ax, static_cast<double>(alpha)) / pow(aw, 1.0 - alpha);
   s = fmin(fmax(s, 1e-5), 1e5);
   smooth[c] = static_cast<float>(s);
-  folded[c] = static_cast<float>((1.0 + static_cast<double>(w[c])) / s - 1.0);
+  if (w != nullptr) folded[c] = static_cast<float>((1.0 + static_cast<double>(w[c])) / s - 1.0);
+}
+
+// ---------------------------------------------------------------------------
+// MLP boundary preparation (offline)
+// ---------------------------------------------------------------------------
+// Rows of gate and up in alternating blocks of SWIGLU_BLOCK: output row r is
+// gate row 16 (r / 32) + r % 32 when r % 32 < 16, else the up row 16 (r / 32)
+// + r % 32 - 16.  Rows are copied as 32-bit words.
+__global__ void __launch_bounds__(256) interleave_rows_kernel(const uint32_t* g, const uint32_t* u,
+                                                              uint32_t* out, size_t I, size_t wpr) {
+  const size_t total = 2 * I * wpr;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t r = i / wpr, w = i - r * wpr;
+    const size_t blk = r / 32, k = r % 32;
+    const uint32_t* src = k < 16 ? g : u;
+    out[i] = src[(16 * blk + (k & 15)) * wpr + w];
+  }
+}
+
+// s_row[i] / smooth[i]: a per-channel scale 1 / smooth folded into the rows of
+// a row-quantised weight (the codes of a row do not change when it is scaled)
+__global__ void __launch_bounds__(256) fold_row_scales_kernel(float* s_row, const float* smooth,
+                                                              int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) s_row[i] = s_row[i] / smooth[i];
 }
 
 }  // namespace convrot
