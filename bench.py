@@ -152,15 +152,20 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 class Linear:
-    def __init__(self, lin, Wq, s_row, group_in):
+    def __init__(self, lin, Wq, s_row, group_in, swiglu=False):
         self.lin = lin
         self.Wq = Wq
         self.s_row = s_row
         self.group_in = group_in
+        self.swiglu = swiglu  # gate/up GEMM whose epilogue writes SiLU(gate) * up
+        self.out_cols = lin.N // 2 if swiglu else lin.N
 
 
 def input_groups(w):
     """Linears that read the same activation share one rotate-quantise call."""
+    if w.mlp:
+        return [{"key": "mlp", "K": w.linears[0].K, "linears": [w.linears[0]]},
+                {"key": "down", "K": w.linears[1].K, "linears": [w.linears[1]]}]
     groups = []
     for lin in w.linears:
         key = {"q_proj": "attn", "k_proj": "attn", "v_proj": "attn", "o_proj": "o",
@@ -174,8 +179,28 @@ def input_groups(w):
     return groups
 
 
+def prepare_mlp(cr, w, dev):
+    """The MLP block's inputs and offline preparation (untimed): SmoothQuant
+    into the norm weight and into up_proj's row scales, interleaved gate/up."""
+    groups = input_groups(w)
+    gu = w.linears[0]
+    x = workloads.activations(w.M, gu.K, dist=w.dist, outlier_count=w.n_outliers(gu.K),
+                              outlier_scale=w.outlier_scale).to(dev)
+    nw = workloads.norm_weight(gu.K).to(dev)
+    Wg, Wu, Wd = (t.to(dev) for t in workloads.mlp_weights(w, device=dev))
+    mlp = cr.ConvRotMLP(Wg, Wu, Wd, norm_w=nw, x_calib=x)
+    del Wg, Wu, Wd
+    # the second group's input is the intermediate H, written by the gate/up GEMM
+    h = torch.empty(w.M, gu.N // 2, dtype=torch.bfloat16, device=dev)
+    layers = [Linear(gu, mlp.Wq_gu, mlp.s_gu, 0, swiglu=True), Linear(w.linears[1], mlp.Wq_d, mlp.s_d, 1)]
+    torch.cuda.synchronize(dev)
+    return groups, [x, h], [mlp.norm_w, None], layers, mlp
+
+
 def prepare(cr, w, dev):
     """Synthetic inputs and offline weight preparation (untimed)."""
+    if w.mlp:
+        return prepare_mlp(cr, w, dev)[:4]
     groups = input_groups(w)
     inputs, norms = [], []
     for gi, g in enumerate(groups):
@@ -215,18 +240,22 @@ def run_ours(args, rank, world, dev):
     groups, inputs, norms, layers = prepare(cr, w, dev)
 
     # copies of the per-step operands so that no step finds its inputs in L2
+    # (the MLP block's H is produced inside the step: one buffer for all copies)
     step_bytes = sum(x.numel() * 2 for x in inputs) + sum(l.Wq.numel() for l in layers)
     copies = 1 if step_bytes > 2 * L2_BYTES else min(8, math.ceil(3 * L2_BYTES / step_bytes))
     if args.copies > 0:
         copies = args.copies
-    x_sets = [inputs] + [[x.clone() for x in inputs] for _ in range(copies - 1)]
+    x_sets = [inputs] + [[x if (w.mlp and gi == 1) else x.clone() for gi, x in enumerate(inputs)]
+                         for _ in range(copies - 1)]
     w_sets = [[(l.Wq, l.s_row) for l in layers]] + \
              [[(l.Wq.clone(), l.s_row.clone()) for l in layers] for _ in range(copies - 1)]
     ws = cr.Workspace(dev.index)
     Xq = [torch.empty(w.M, g["K"], dtype=torch.int8, device=dev) for g in groups]
     st = [torch.empty(w.M, dtype=torch.float32, device=dev) for g in groups]
-    Ys = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16, device=dev) for l in layers]
+    Ys = [inputs[1] if l.swiglu else torch.empty(w.M, l.out_cols, dtype=torch.bfloat16, device=dev)
+          for l in layers]
     linear = cr.convrot_int8_linear if w.weight_bits == 8 else cr.convrot_w4a8_linear
+    swiglu = cr.convrot_int8_linear_swiglu if w.weight_bits == 8 else cr.convrot_w4a8_linear_swiglu
 
     stream = torch.cuda.current_stream(dev)
     n_k1 = len(groups)
@@ -238,7 +267,16 @@ def run_ours(args, rank, world, dev):
     def launch_k2(c, li):
         l = layers[li]
         Wq, s_row = w_sets[c][li]
-        linear(Xq[l.group_in], st[l.group_in], Wq, s_row, out=Ys[li], workspace=ws)
+        (swiglu if l.swiglu else linear)(Xq[l.group_in], st[l.group_in], Wq, s_row, out=Ys[li],
+                                         workspace=ws)
+
+    # launch order of one step: every rotate-quantise, then every GEMM; the
+    # MLP block is a chain (x -> gate/up -> H -> down)
+    order = ([("k1", 0), ("k2", 0), ("k1", 1), ("k2", 1)] if w.mlp else
+             [("k1", gi) for gi in range(len(groups))] + [("k2", li) for li in range(len(layers))])
+
+    def launch(c, kind, idx):
+        (launch_k1 if kind == "k1" else launch_k2)(c, idx)
 
     # Graph mode (default): the W warm-up steps and the K timed steps are each
     # captured as ONE CUDA graph of the same ABI calls (step i reads input copy
@@ -249,17 +287,13 @@ def run_ours(args, rank, world, dev):
     # between two kernels inside a graph costs ~5 us on this GPU, so kernels
     # are not bracketed one by one.)  --eager issues the same calls directly.
     for c in range(copies):  # eager warm-up: encodes and caches every tensor map
-        for gi in range(n_k1):
-            launch_k1(c, gi)
-        for li in range(n_k2):
-            launch_k2(c, li)
+        for kind, idx in order:
+            launch(c, kind, idx)
     torch.cuda.synchronize(dev)
 
     def step(i):
-        for gi in range(n_k1):
-            launch_k1(i % copies, gi)
-        for li in range(n_k2):
-            launch_k2(i % copies, li)
+        for kind, idx in order:
+            launch(i % copies, kind, idx)
 
     def k1_only(i):
         for gi in range(n_k1):
@@ -350,8 +384,9 @@ def run_ours(args, rank, world, dev):
     tokens = w.M * args.steps * world
     ops = w.ops() * args.steps * world
     secs = elapsed_ms / 1e3
-    k1_bytes = sum(w.M * g["K"] * 3 + 4 * w.M + (4 * g["K"] if w.norm else 0) for g in groups)
-    k2_bytes = sum(w.M * l.lin.K + l.Wq.numel() + 2 * w.M * l.lin.N + 4 * (w.M + l.lin.N)
+    k1_bytes = sum(w.M * g["K"] * 3 + 4 * w.M + (4 * g["K"] if norms[gi] is not None else 0)
+                   for gi, g in enumerate(groups))
+    k2_bytes = sum(w.M * l.lin.K + l.Wq.numel() + 2 * w.M * l.out_cols + 4 * (w.M + l.lin.N)
                    for l in layers)
     k2_ops = w.ops()
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -392,6 +427,8 @@ def run_ours(args, rank, world, dev):
             "workload": args.workload, "M": w.M,
             "linears": [[l.name, l.N, l.K] for l in w.linears], "layers": w.layers,
             "weight_bits": w.weight_bits, "group": 256, "rmsnorm": w.norm,
+            **({"block": "down(SiLU(gate(x)) * up(x)); gate/up as one GEMM with the SwiGLU epilogue"}
+               if w.mlp else {}),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "launch": ("eager ABI calls" if timed_graph is None else
                        "the K timed steps' ABI calls captured as one CUDA graph, replayed once"),
@@ -427,20 +464,38 @@ def run_ours(args, rank, world, dev):
 def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
     """Same metric through the public API with pinned host buffers: each step
     copies its activations host->device and its outputs device->host."""
-    host_x = [x.cpu().pin_memory() for x in inputs]
-    host_y = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16).pin_memory() for l in layers]
     ws = cr.Workspace(dev.index)
     linear = cr.convrot_int8_linear if w.weight_bits == 8 else cr.convrot_w4a8_linear
     stream = torch.cuda.current_stream(dev)
     steps = max(5, min(args.steps, 50))
+    if w.mlp:
+        # the block's input comes from the host and its output goes back; H
+        # stays on the device between the two GEMMs
+        host_x = [inputs[0].cpu().pin_memory()]
+        host_y = [torch.empty(w.M, layers[1].out_cols, dtype=torch.bfloat16).pin_memory()]
+        gu, down = layers
+        swiglu = cr.convrot_int8_linear_swiglu if w.weight_bits == 8 else cr.convrot_w4a8_linear_swiglu
 
-    def step():
+        def step():
+            x = host_x[0].to(dev, non_blocking=True)
+            Xq, s_tok = cr.convrot_rotate_quant_act(x, 256, norms[0], 1e-6)
+            H = swiglu(Xq, s_tok, gu.Wq, gu.s_row, workspace=ws)
+            Hq, s_h = cr.convrot_rotate_quant_act(H, 256, None, 1e-6)
+            host_y[0].copy_(linear(Hq, s_h, down.Wq, down.s_row, workspace=ws), non_blocking=True)
+    else:
+        host_x = [x.cpu().pin_memory() for x in inputs]
+        host_y = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16).pin_memory() for l in layers]
+        step = None
+
+    def layer_step():
         xs = [h.to(dev, non_blocking=True) for h in host_x]
         qs = [cr.convrot_rotate_quant_act(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
         for li, l in enumerate(layers):
             Y = linear(qs[l.group_in][0], qs[l.group_in][1], l.Wq, l.s_row, workspace=ws)
             host_y[li].copy_(Y, non_blocking=True)
 
+    if step is None:
+        step = layer_step
     for _ in range(3):
         step()
     torch.cuda.synchronize(dev)
@@ -467,6 +522,8 @@ def oracle_step_runner(w, sample_tokens):
     """Prepares the oracle's weights (untimed) and returns a callable that runs
     the oracle's per-token path on `sample_tokens` tokens of the workload."""
     from oracle import convrot_ref as ref
+    if w.mlp:
+        return oracle_mlp_runner(ref, w, sample_tokens)
     groups = input_groups(w)
     xs, nws, preps = [], [], []
     for g in groups:
@@ -495,6 +552,34 @@ def oracle_step_runner(w, sample_tokens):
                 ref.int8_linear(Xq, s_tok, Wq, s_row)
             else:
                 ref.w4a8_linear(Xq, s_tok, packed, s_row)
+    return run
+
+
+def oracle_mlp_runner(ref, w, sample_tokens):
+    """The MLP block through the oracle: calibration and weight preparation on
+    the sample (untimed), then norm + rotate-quantise, gate/up with SiLU(gate)
+    * up, rotate-quantise of H and down_proj per call."""
+    gu = w.linears[0]
+    x, _, nw = workloads.workload_inputs(w, gu, M=min(w.M, max(sample_tokens, 1)))
+    x64 = x.float().double().numpy()[:sample_tokens]
+    Wg, Wu, Wd = (t.float().double().numpy() for t in workloads.mlp_weights(w))
+    sc, wf = ref.smoothquant_scales(x64, nw.double().numpy(), 1e-6, np.concatenate([Wg, Wu]))
+    qg, sg, _ = ref.quantize_weight(Wg, 256, sc)
+    qu, su, _ = ref.quantize_weight(Wu, 256, sc)
+    del Wg, Wu
+    qgu = ref.interleave_gate_up(qg, qu)
+    Xq, st, _ = ref.rotate_quant_act(x64, 256, wf, 1e-6)
+    h0, _, _ = ref.swiglu_linear(Xq, st, qgu, ref.interleave_gate_up(sg, su))
+    sd = ref.smoothquant_scales_of(h0, Wd)
+    sgu = ref.interleave_gate_up(sg, ref.fold_smooth_into_rows(su, sd))
+    qd, sdr, _ = ref.quantize_weight(Wd, 256, sd)
+    del Wd
+
+    def run():
+        Xq, st, _ = ref.rotate_quant_act(x64, 256, wf, 1e-6)
+        hb, _, _ = ref.swiglu_linear(Xq, st, qgu, sgu)
+        Hq, sh, _ = ref.rotate_quant_act(hb, 256)
+        ref.int8_linear(Hq, sh, qd, sdr)
     return run
 
 

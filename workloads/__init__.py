@@ -14,4 +14,5 @@ from .synthetic import (  # noqa: F401
     norm_weight,
     outlier_channels,
     workload_inputs,
+    mlp_weights,
 )

@@ -111,6 +111,10 @@ class Workload:
     norm: bool = False          # RMSNorm with folded SmoothQuant scale before the linear
     weight_bits: int = 8        # 8 = int8 codes, 4 = packed signed 4-bit codes
     layers: int = 1
+    # MLP block down(SiLU(gate(x)) * up(x)): linears[0] is the fused gate/up
+    # projection (N = 2 I rows, gate and up interleaved), linears[1] down_proj,
+    # whose input is the block's intermediate H instead of fresh activations
+    mlp: bool = False
 
     def n_outliers(self, K: int) -> int:
         if self.outlier_count:
@@ -151,11 +155,26 @@ WORKLOADS = {
     **{f"gate_up_m{m}": Workload(f"gate_up_m{m}", m, (Linear("gate_up", 24576, 4096),),
                                  outlier_frac=0.01, outlier_scale=20.0)
        for m in (1, 16, 128, 1024, 8192)},
+    # the decoder layer's MLP block as one chain: RMSNorm + rotate-quantise,
+    # gate/up GEMM with the SiLU(gate) * up epilogue, rotate-quantise of H,
+    # down_proj; SmoothQuant folded into the norm and into up_proj's rows
+    "mlp_block_m2048": Workload("mlp_block_m2048", 2048,
+                                (Linear("gate_up", 24576, 4096), Linear("down_proj", 4096, 12288)),
+                                outlier_frac=0.005, outlier_scale=20.0, norm=True, mlp=True),
     # int4-weight variant over 36 decoder layers
     "w4a8_36_layers_m4096": Workload("w4a8_36_layers_m4096", 4096, _DECODER,
                                      outlier_frac=0.01, outlier_scale=20.0,
                                      weight_bits=4, layers=36),
 }
+
+
+def mlp_weights(w: Workload, device="cpu"):
+    """(Wg [I, H], Wu [I, H], Wd [H, I]) bf16 of an MLP-block workload, seeds
+    SEED_W, SEED_W + 1 and SEED_W + 2."""
+    gu, down = w.linears
+    I, H = gu.N // 2, gu.K
+    return (weight(I, H, seed=SEED_W, device=device), weight(I, H, seed=SEED_W + 1, device=device),
+            weight(H, I, seed=SEED_W + 2, device=device))
 
 
 def workload_inputs(w: Workload, lin: Linear, *, M: Optional[int] = None, layer: int = 0,
