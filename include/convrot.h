@@ -14,7 +14,9 @@
  *  - "Qwen3-VL-8B-Heretic-1.3.0 - INT8 ConvRot (ComfyUI)", "Quantization
  *    metadata": convrot true, convrot_groupsize 256, per_row true.
  *  - "Qwen3-VL 8B - INT8 ConvRot", "Layer and group selection": widths the
- *    group does not divide fall back to plain row-wise INT8 (group = 0 here).
+ *    group does not divide fall back to plain row-wise INT8 (group = 0 here);
+ *    the vision tower's widths 1152 and 4304 use 16-point groups instead
+ *    ("Original version conversion": vision ConvRot group size 16).
  *  - "MossInt4", "Format": the convrot_w4a4 layout (signed 4-bit codes, two
  *    per byte, one F32 scale per row from a per-row clip search, 8-bit
  *    activations).
@@ -64,7 +66,7 @@ typedef enum {
   CONVROT_ERR_NULL = 1,            /* a required pointer is NULL */
   CONVROT_ERR_SHAPE = 2,           /* a size is negative, too large or not a required multiple */
   CONVROT_ERR_ALIGN = 3,           /* a pointer is not aligned as required */
-  CONVROT_ERR_UNSUPPORTED = 4,     /* e.g. a group size other than 0 or 256 */
+  CONVROT_ERR_UNSUPPORTED = 4,     /* e.g. a group size other than 0, 16 or 256 */
   CONVROT_ERR_CUDA = 5,            /* a CUDA runtime or driver call failed */
   CONVROT_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on a bounded wait */
   CONVROT_ERR_WORKSPACE = 7        /* workspace missing or smaller than required */
@@ -116,7 +118,8 @@ convrot_status convrot_selftest_wait_timeout(uint32_t limit_cycles, convrot_stre
  * col_scale fp32 [K] or NULL    in   SmoothQuant scale s folded into the weight
  * Wq     int8 [N, K]            out
  * s_row  fp32 [N]               out
- * group  256 (K % 256 == 0) or 0 (K % 16 == 0)
+ * group  256 (K % 256 == 0), 16 (K % 16 == 0; H = H_16 / 4 per 16 columns)
+ *        or 0 (no rotation, K % 16 == 0)
  */
 convrot_status convrot_quantize_weight(const void* W, int N, int K, int group,
                                        const float* col_scale, int8_t* Wq, float* s_row,
@@ -132,7 +135,8 @@ convrot_status convrot_quantize_weight(const void* W, int N, int K, int group,
  * Wq4    uint8 [N, K/2]  out   byte j of a row holds code 2j in bits 0-3 and
  *                              code 2j+1 in bits 4-7, two's complement
  * s_row  fp32 [N]        out
- * K % 32 == 0 (and K % 256 == 0 when group == 256); 1 <= clip_steps <= 64.
+ * group 256, 16 or 0 as convrot_quantize_weight; K % 32 == 0 (and K % 256 == 0
+ * when group == 256); 1 <= clip_steps <= 64.
  */
 convrot_status convrot_quantize_weight_w4(const void* W, int N, int K, int group,
                                           const float* col_scale, float clip_lo,
@@ -174,7 +178,7 @@ convrot_status convrot_smoothquant_calibrate(const void* x, int M, int K, const 
  *   s_tok[m] = max_k |v[m,k]| / 127           (0 for an all-zero row)
  *   Xq[m,k]  = clamp(rint(v[m,k] / s_tok[m]), -127, 127), round-half-even
  * x bf16 [M, K] in, norm_w fp32 [K] or NULL in, Xq int8 [M, K] out,
- * s_tok fp32 [M] out.  group 256 (K % 256 == 0) or 0 (K % 16 == 0).
+ * s_tok fp32 [M] out.  group 256 (K % 256 == 0), 16 or 0 (K % 16 == 0).
  * The rotation is computed in fp32 registers; codes can differ from an exact
  * evaluation only where v / s_tok lies within fp32 rounding of a tie.
  */

@@ -58,8 +58,11 @@ def test_validation_before_any_launch(lib):
     assert lib.convrot_rotate_quant_act(A, 4, 512, 128, None, 1e-6, A, A, None) == 4
     # K not a multiple of the group
     assert lib.convrot_rotate_quant_act(A, 4, 384, 256, None, 1e-6, A, A, None) == 2
-    # K not a multiple of 16 with group 0
+    # K not a multiple of 16 with group 0 or 16
     assert lib.convrot_rotate_quant_act(A, 4, 40, 0, None, 1e-6, A, A, None) == 2
+    assert lib.convrot_rotate_quant_act(A, 4, 40, 16, None, 1e-6, A, A, None) == 2
+    # int4 weights need K % 32 also with group 16
+    assert lib.convrot_quantize_weight_w4(A, 4, 4304, 16, None, 0.8, 1.0, 21, A, A, None) == 2
     # null pointers
     assert lib.convrot_rotate_quant_act(None, 4, 512, 256, None, 1e-6, A, A, None) == 1
     assert lib.convrot_quantize_weight(A, 4, 512, 256, None, None, A, None) == 1

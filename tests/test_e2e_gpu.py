@@ -197,3 +197,12 @@ def test_convrot_linear_object(cr):
         yb, _, _ = _reference(x, W, None, bits, xq.cpu().numpy(),
                               (wq, layer.s_row.cpu().double().numpy()))
         _assert_close(Y, yb, f"ConvRotLinear int{bits}")
+
+
+@pytest.mark.parametrize("K,N", [(1152, 4304), (4304, 1152)])
+def test_group16_vision_linear_all_outputs(cr, K, N):
+    # a vision-tower linear with 16-point ConvRot groups ("Qwen3-VL 8B - INT8
+    # ConvRot", "Layer and group selection"): widths 1152 and 4304
+    x = workloads.activations(64, K, outlier_count=K // 100, seed=K)
+    W = workloads.weight(N, K, seed=N)
+    _full(cr, x, W, None, 8, group=16, what=f"group-16 linear {K}->{N}")

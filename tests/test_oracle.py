@@ -102,6 +102,33 @@ def test_rotation_brute_force_tiny():
             assert got[256 * g + i] == s
 
 
+def test_hadamard_16_for_the_vision_group():
+    # "Qwen3-VL 8B - INT8 ConvRot", "Layer and group selection": group size 16
+    # for vision widths 1152 and 4304, which 256 does not divide but 16 does
+    h = ref.hadamard(16)
+    assert np.array_equal(h @ h.T, np.eye(16)) and np.array_equal(h, h.T)
+    for i in range(16):
+        for j in range(16):
+            assert h[i, j] * 4.0 == _popsign(i, j)
+    assert 1152 % 256 and 4304 % 256 and not 1152 % 16 and not 4304 % 16
+
+
+def test_rotation_group16_brute_force():
+    rng = np.random.default_rng(4)
+    x = rng.integers(-4, 5, size=(2, 48)).astype(np.float64)
+    got = ref.rotate_groups(x, 16)
+    for r in range(2):
+        for g in range(3):
+            for i in range(16):
+                s = sum(x[r, 16 * g + j] * _popsign(i, j) for j in range(16)) / 4
+                assert got[r, 16 * g + i] == s
+    # products survive the rotation as for 256-groups
+    W = rng.standard_normal((5, 1152))
+    xx = rng.standard_normal((3, 1152))
+    np.testing.assert_allclose(ref.rotate_groups(xx, 16) @ ref.rotate_groups(W, 16).T, xx @ W.T,
+                               rtol=1e-12, atol=1e-12)
+
+
 def test_group_zero_is_plain_rowwise():
     rng = np.random.default_rng(2)
     x = rng.standard_normal((3, 48))

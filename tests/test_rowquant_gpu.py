@@ -67,6 +67,16 @@ def test_act_group0_plain_rowwise(cr, K):
     _check_act(cr, x, 0, workloads.norm_weight(K))
 
 
+@pytest.mark.parametrize("M", [1, 37, 300])
+@pytest.mark.parametrize("K", [16, 48, 1152, 4096, 4304])
+@pytest.mark.parametrize("norm", [False, True])
+def test_act_group16(cr, M, K, norm):
+    # 16-point groups for widths 256 does not divide ("Qwen3-VL 8B - INT8
+    # ConvRot", "Layer and group selection": vision widths 1152 and 4304)
+    x = workloads.activations(M, K, outlier_count=max(1, K // 100), seed=M + K)
+    _check_act(cr, x, 16, workloads.norm_weight(K) if norm else None)
+
+
 @pytest.mark.parametrize("K", [16640, 32768, 131072])
 def test_act_streaming_path_large_K(cr, K):
     # rows wider than one CTA team are processed in two passes
@@ -138,16 +148,17 @@ def test_act_full_size_gate_up_sampled(cr):
 
 
 # ---------------------------------------------------------------- weights
-@pytest.mark.parametrize("N,K", [(8, 256), (24, 512), (136, 4096), (40, 12288), (16, 16640)])
+@pytest.mark.parametrize("N,K,group", [(8, 256, 256), (24, 512, 256), (136, 4096, 256), (40, 12288, 256),
+                                       (16, 16640, 256), (24, 1152, 16), (40, 4304, 16), (8, 16640, 16)])
 @pytest.mark.parametrize("colscale", [False, True])
-def test_weight_int8(cr, N, K, colscale):
+def test_weight_int8(cr, N, K, group, colscale):
     W = workloads.weight(N, K, seed=N + K)
     cs = (torch.rand(K, generator=torch.Generator().manual_seed(5)) * 4 + 0.25) if colscale else None
-    Wq, s_row = cr.convrot_quantize_weight(W.cuda(), 256, None if cs is None else cs.cuda())
+    Wq, s_row = cr.convrot_quantize_weight(W.cuda(), group, None if cs is None else cs.cuda())
     torch.cuda.synchronize()
-    q_ref, s_ref32, Wr = ref.quantize_weight(_f64(W), 256, None if cs is None else cs.double().numpy())
+    q_ref, s_ref32, Wr = ref.quantize_weight(_f64(W), group, None if cs is None else cs.double().numpy())
     s_ref = np.max(np.abs(Wr), axis=1) / 127.0
-    ratio, _ = _tol.row_error(Wr, 256, colscale)
+    ratio, _ = _tol.row_error(Wr, group, colscale)
     sg = s_row.cpu().double().numpy()
     assert np.all(np.abs(sg - s_ref) <= _tol.scale_rel_tol(ratio, False) * s_ref)
     _tol.check_codes(Wq.cpu().numpy(), q_ref, Wr / s_ref[:, None], _tol.int8_code_window(ratio))
@@ -204,6 +215,11 @@ def _w4_check(cr, W, group=256, cs=None, clip=(0.80, 1.00, 21)):
 @pytest.mark.parametrize("N,K", [(8, 256), (40, 512), (64, 4096), (16, 12288), (8, 16640)])
 def test_weight_int4_clip_search(cr, N, K):
     _w4_check(cr, workloads.weight(N, K, seed=N * K))
+
+
+@pytest.mark.parametrize("N,K", [(24, 1152), (8, 4320)])
+def test_weight_int4_group16(cr, N, K):
+    _w4_check(cr, workloads.weight(N, K, seed=N + 3 * K), group=16)
 
 
 def test_weight_int4_group0_colscale_and_grid(cr):

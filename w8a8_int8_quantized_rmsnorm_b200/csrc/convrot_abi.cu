@@ -187,9 +187,9 @@ convrot_status launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t sme
   return launch_status();
 }
 
-template <bool ROT, int PRE, int QK, bool RES>
+template <int GRP, int PRE, int QK, bool RES>
 convrot_status launch_rowquant_t(const RowQuantArgs& a, int threads, cudaStream_t st) {
-  auto k = rowquant_kernel<ROT, PRE, QK, RES>;
+  auto k = rowquant_kernel<GRP, PRE, QK, RES>;
   const DeviceInfo d = current_device();
   // occupancy per (device, block size in warps), computed once
   static std::atomic<int> occ[64][33];
@@ -205,26 +205,30 @@ convrot_status launch_rowquant_t(const RowQuantArgs& a, int threads, cudaStream_
   return launch_pdl(k, dim3(grid), dim3(threads), 0, st, 1, a);
 }
 
+template <int GRP, int PRE, int QK>
+convrot_status launch_rowquant_grp(const RowQuantArgs& a, const RowPlan& p, cudaStream_t st) {
+  const int threads = p.team * p.rows_per_cta;
+  return p.resident ? launch_rowquant_t<GRP, PRE, QK, true>(a, threads, st)
+                    : launch_rowquant_t<GRP, PRE, QK, false>(a, threads, st);
+}
+
+// group: 256, 16 or 0 (no rotation)
 template <int PRE, int QK>
-convrot_status launch_rowquant_pre(RowQuantArgs& a, bool rot, cudaStream_t st) {
+convrot_status launch_rowquant_pre(RowQuantArgs& a, int group, cudaStream_t st) {
   const RowPlan p = plan_rows(a.K);
   a.team = p.team;
   a.rows_per_cta = p.rows_per_cta;
   a.passes = p.passes;
-  const int threads = p.team * p.rows_per_cta;
-  if (rot) {
-    return p.resident ? launch_rowquant_t<true, PRE, QK, true>(a, threads, st)
-                      : launch_rowquant_t<true, PRE, QK, false>(a, threads, st);
-  }
-  return p.resident ? launch_rowquant_t<false, PRE, QK, true>(a, threads, st)
-                    : launch_rowquant_t<false, PRE, QK, false>(a, threads, st);
+  if (group == 256) return launch_rowquant_grp<256, PRE, QK>(a, p, st);
+  if (group == 16) return launch_rowquant_grp<16, PRE, QK>(a, p, st);
+  return launch_rowquant_grp<0, PRE, QK>(a, p, st);
 }
 
 // TMA-fed activation kernel: teams of rowquant's layout, one CTA per SM, a
 // ring of stages of `rows` token rows each.
-template <bool ROT, bool NORM>
+template <int GRP, bool NORM>
 convrot_status launch_actquant_t(ActArgs a, cudaStream_t st) {
-  auto k = actquant_kernel<ROT, NORM>;
+  auto k = actquant_kernel<GRP, NORM>;
   const DeviceInfo d = current_device();
   const int dyn = a.wsm_bytes + a.stages * a.rows * a.K * 2;
   static std::atomic<int> configured[64];
@@ -259,7 +263,7 @@ bool plan_actquant(int K, ActArgs& a) {
 }
 
 convrot_status check_group(int group, int K, int multiple) {
-  if (group != 0 && group != 256) return CONVROT_ERR_UNSUPPORTED;
+  if (group != 0 && group != 16 && group != 256) return CONVROT_ERR_UNSUPPORTED;
   if (K <= 0 || K > CONVROT_MAX_K) return CONVROT_ERR_SHAPE;
   if (K % multiple) return CONVROT_ERR_SHAPE;
   if (group == 256 && K % 256) return CONVROT_ERR_SHAPE;
@@ -664,9 +668,8 @@ convrot_status convrot_quantize_weight(const void* W, int N, int K, int group,
   a.scale = s_row;
   a.rows = N;
   a.K = K;
-  const bool rot = group == 256;
-  return col_scale ? launch_rowquant_pre<PRE_COLSCALE, QK_INT8>(a, rot, as_cuda(stream))
-                   : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, rot, as_cuda(stream));
+  return col_scale ? launch_rowquant_pre<PRE_COLSCALE, QK_INT8>(a, group, as_cuda(stream))
+                   : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, group, as_cuda(stream));
 }
 
 convrot_status convrot_quantize_weight_w4(const void* W, int N, int K, int group,
@@ -697,9 +700,8 @@ convrot_status convrot_quantize_weight_w4(const void* W, int N, int K, int group
     a.clip_step = static_cast<float>((static_cast<double>(clip_hi) - clip_lo) / (clip_steps - 1));
   }
   a.clip_steps = clip_steps;
-  const bool rot = group == 256;
-  return col_scale ? launch_rowquant_pre<PRE_COLSCALE, QK_INT4>(a, rot, as_cuda(stream))
-                   : launch_rowquant_pre<PRE_NONE, QK_INT4>(a, rot, as_cuda(stream));
+  return col_scale ? launch_rowquant_pre<PRE_COLSCALE, QK_INT4>(a, group, as_cuda(stream))
+                   : launch_rowquant_pre<PRE_NONE, QK_INT4>(a, group, as_cuda(stream));
 }
 
 convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
@@ -713,7 +715,6 @@ convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
   if (!x || !Xq || !s_tok) return CONVROT_ERR_NULL;
   if (!aligned(x, 16) || !aligned(Xq, 16) || !aligned(s_tok, 4)) return CONVROT_ERR_ALIGN;
   if (norm_w && !aligned(norm_w, 16)) return CONVROT_ERR_ALIGN;
-  const bool rot = group == 256;
   ActArgs q{};
   q.x = static_cast<const uint16_t*>(x);
   q.norm_w = norm_w;
@@ -729,8 +730,11 @@ convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
     }
     if (q.stages >= 2) {
       cudaStream_t st = as_cuda(stream);
-      if (rot) return norm_w ? launch_actquant_t<true, true>(q, st) : launch_actquant_t<true, false>(q, st);
-      return norm_w ? launch_actquant_t<false, true>(q, st) : launch_actquant_t<false, false>(q, st);
+      if (group == 256)
+        return norm_w ? launch_actquant_t<256, true>(q, st) : launch_actquant_t<256, false>(q, st);
+      if (group == 16)
+        return norm_w ? launch_actquant_t<16, true>(q, st) : launch_actquant_t<16, false>(q, st);
+      return norm_w ? launch_actquant_t<0, true>(q, st) : launch_actquant_t<0, false>(q, st);
     }
   }
   RowQuantArgs a{};
@@ -741,8 +745,8 @@ convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
   a.rows = M;
   a.K = K;
   a.eps = eps;
-  return norm_w ? launch_rowquant_pre<PRE_NORM, QK_INT8>(a, rot, as_cuda(stream))
-                : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, rot, as_cuda(stream));
+  return norm_w ? launch_rowquant_pre<PRE_NORM, QK_INT8>(a, group, as_cuda(stream))
+                : launch_rowquant_pre<PRE_NONE, QK_INT8>(a, group, as_cuda(stream));
 }
 
 convrot_status convrot_smoothquant_calibrate(const void* x, int M, int K, const float* norm_w,

@@ -196,22 +196,33 @@ __device__ __forceinline__ void lane_swap(float (&v)[64], int h, int m, int lane
   }
 }
 
-// Unnormalised 256-point Walsh-Hadamard transform of one group held by four
-// lanes (natural Sylvester order), or only the data movement when ROT is off.
-template <bool ROT>
+// Unnormalised Walsh-Hadamard transform (natural Sylvester order) of the
+// GRP-element groups within the 256 elements held by four lanes: GRP = 256
+// runs all eight butterfly stages, GRP = 16 the stages of element bits 0-3,
+// GRP = 0 only the data movement.
+template <int GRP>
 __device__ __forceinline__ void rq_transform(float (&v)[64], int lane) {
-  if (ROT) {
+  static_assert(GRP == 0 || GRP == 16 || GRP == 256, "group size 0, 16 or 256");
+  if (GRP) {
     butterfly(v, 1);   // element bit 0
     butterfly(v, 2);   // element bit 1
     butterfly(v, 4);   // element bit 2
+  }
+  if (GRP == 256) {
     butterfly(v, 8);   // element bit 5
     butterfly(v, 16);  // element bit 6
     butterfly(v, 32);  // element bit 7
   }
   lane_swap(v, 8, 1, lane);  // register bit 3 <-> element bit 3
-  if (ROT) butterfly(v, 8);
+  if (GRP) butterfly(v, 8);
   lane_swap(v, 16, 2, lane);  // register bit 4 <-> element bit 4
-  if (ROT) butterfly(v, 16);
+  if (GRP == 256) butterfly(v, 16);
+}
+
+// 1 / sqrt(GRP): the normalisation of H_GRP, applied to the per-row scale.
+template <int GRP>
+__host__ __device__ constexpr double group_norm() {
+  return GRP == 256 ? 1.0 / 16.0 : (GRP == 16 ? 1.0 / 4.0 : 1.0);
 }
 
 __device__ __forceinline__ float rq_absmax(const float (&v)[64]) {
@@ -287,7 +298,7 @@ __device__ __forceinline__ void rq_store_int4(const RowQuantArgs& a, uint8_t* ro
   }
 }
 
-template <bool ROT, int PRE, int QK, bool RESIDENT>
+template <int GRP, int PRE, int QK, bool RESIDENT>
 __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
   __shared__ float s_max[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
   __shared__ double s_sum[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
@@ -315,13 +326,13 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
     if (RESIDENT) {
       const int g = t >> 2;
       rq_load<PRE>(a, src_row, g, L, row_ok && g < G, v, sq);
-      rq_transform<ROT>(v, lane);
+      rq_transform<GRP>(v, lane);
       amax = rq_absmax(v);
     } else {
       for (int p = 0; p < a.passes; ++p) {
         const int g = (t + p * a.team) >> 2;
         rq_load<PRE>(a, src_row, g, L, row_ok && g < G, v, sq);
-        rq_transform<ROT>(v, lane);
+        rq_transform<GRP>(v, lane);
         amax = fmaxf(amax, rq_absmax(v));
       }
     }
@@ -344,9 +355,9 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
       }
     }
 
-    // fp64 per-row scale: absmax of the unnormalised transform, times 1/16
-    // for H = H_256 / 16, times r for the RMSNorm.
-    double rowfac = ROT ? 1.0 / 16.0 : 1.0;
+    // fp64 per-row scale: absmax of the unnormalised transform, times
+    // 1/sqrt(GRP) for the normalised Hadamard, times r for the RMSNorm.
+    double rowfac = group_norm<GRP>();
     if (PRE == PRE_NORM) {
       const double ms = sumsq / static_cast<double>(a.K);
       rowfac *= 1.0 / sqrt(ms + static_cast<double>(a.eps));
@@ -365,7 +376,7 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
           const int g = (t + p * a.team) >> 2;
           float sq2 = 0.f;
           rq_load<PRE>(a, src_row, g, L, row_ok && g < G, v, sq2);
-          rq_transform<ROT>(v, lane);
+          rq_transform<GRP>(v, lane);
           rq_store_int8(a, dst_row, g, L, row_ok && g < G, v, inv);
         }
       }
@@ -384,7 +395,7 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
               const int g = (t + p * a.team) >> 2;
               float sq2 = 0.f;
               rq_load<PRE>(a, src_row, g, L, row_ok && g < G, v, sq2);
-              rq_transform<ROT>(v, lane);
+              rq_transform<GRP>(v, lane);
               err += rq_sse_int4(v, s);
             }
           }
@@ -409,7 +420,7 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
           const int g = (t + p * a.team) >> 2;
           float sq2 = 0.f;
           rq_load<PRE>(a, src_row, g, L, row_ok && g < G, v, sq2);
-          rq_transform<ROT>(v, lane);
+          rq_transform<GRP>(v, lane);
           rq_store_int4(a, dst_row, g, L, row_ok && g < G, v, best_s);
         }
       }
@@ -578,7 +589,9 @@ __device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm
   sq += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
 }
 
-// Unnormalised FWHT-256 of the group held by four lanes, in place.
+// Unnormalised FWHT of the GRP-element groups (256 or 16) within the 256
+// elements held by four lanes, in place.
+template <int GRP>
 __device__ __forceinline__ void act3_fwht(uint64_t (&v)[32], int lane) {
   // element bit 0: inside each pair
 #pragma unroll
@@ -586,9 +599,10 @@ __device__ __forceinline__ void act3_fwht(uint64_t (&v)[32], int lane) {
     const float x = f2_lo(v[p]), y = f2_hi(v[p]);
     v[p] = f2_pack(x + y, x - y);
   }
-  // element bits 1, 2, 5, 6, 7: between pairs (pair-index bits 0..4)
+  // element bits 1, 2 (and 5, 6, 7 for 256-point groups): between pairs
+  // (pair-index bits 0..4)
 #pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
+  for (int m = 1; m < (GRP == 256 ? 32 : 4); m <<= 1) {
 #pragma unroll
     for (int p = 0; p < 32; ++p) {
       if (!(p & m)) {
@@ -598,10 +612,10 @@ __device__ __forceinline__ void act3_fwht(uint64_t (&v)[32], int lane) {
       }
     }
   }
-  // element bits 3, 4: between lanes (lane bits 0, 1).  The lane whose bit is
-  // clear keeps x + partner, the other partner - x.
+  // element bits 3 (and 4): between lanes (lane bits 0, 1).  The lane whose
+  // bit is clear keeps x + partner, the other partner - x.
 #pragma unroll
-  for (int lm = 1; lm <= 2; lm <<= 1) {
+  for (int lm = 1; lm <= (GRP == 256 ? 2 : 1); lm <<= 1) {
     const float sg = (lane & lm) ? -1.0f : 1.0f;
     const uint64_t s2 = f2_pack(sg, sg);
 #pragma unroll
@@ -648,8 +662,10 @@ __device__ __forceinline__ void act3_store(int8_t* row, int K, int g, int L, boo
   }
 }
 
-template <bool ROT, bool NORM>
+template <int GRP, bool NORM>
 __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
+  // K is a multiple of 256 for 256-point groups: no per-element bounds checks
+  constexpr bool WHOLE = GRP == 256;
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
   __shared__ float s_max[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
   __shared__ double s_sum[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
@@ -741,10 +757,10 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
         reinterpret_cast<const uint16_t*>(ring + s * stage_bytes) + static_cast<size_t>(slot) * a.K;
     uint64_t v[32];
     float sq = 0.f;
-    act3_load<NORM, ROT>(srow, wsm, a.K, g, L, row_ok && g < G, v, sq);
+    act3_load<NORM, WHOLE>(srow, wsm, a.K, g, L, row_ok && g < G, v, sq);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);  // stage read: the producer may refill it
-    if (ROT) act3_fwht(v, lane);
+    if (GRP) act3_fwht<GRP>(v, lane);
     float amax = act3_absmax(v);
     double sumsq = static_cast<double>(sq);
     red.reduce(amax, sumsq);
@@ -763,11 +779,11 @@ __global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
     const float inv = amax > 0.f ? 127.0f / amax : 0.0f;
     if (row_ok && t == 0) {
       // the per-row scale is needed by one thread only
-      double rowfac = ROT ? 1.0 / 16.0 : 1.0;
+      double rowfac = group_norm<GRP>();
       if (NORM) rowfac *= 1.0 / sqrt(sumsq / static_cast<double>(a.K) + static_cast<double>(a.eps));
       a.s_tok[row] = amax > 0.f ? static_cast<float>(static_cast<double>(amax) * rowfac / 127.0) : 0.0f;
     }
-    act3_store<ROT>(a.xq + static_cast<size_t>(row_ok ? row : 0) * a.K, a.K, g, L, row_ok && g < G,
+    act3_store<WHOLE>(a.xq + static_cast<size_t>(row_ok ? row : 0) * a.K, a.K, g, L, row_ok && g < G,
                     v, inv);
   }
 }
