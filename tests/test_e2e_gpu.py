@@ -206,3 +206,38 @@ def test_group16_vision_linear_all_outputs(cr, K, N):
     x = workloads.activations(64, K, outlier_count=K // 100, seed=K)
     W = workloads.weight(N, K, seed=N)
     _full(cr, x, W, None, 8, group=16, what=f"group-16 linear {K}->{N}")
+
+
+@pytest.mark.parametrize("bits,group,K", [(8, 256, 4096), (4, 256, 1024), (8, 16, 1152)])
+def test_checkpoint_round_trip_runs_the_same_layer(cr, tmp_path, bits, group, K):
+    # a layer prepared on the GPU, written as a comfy_quant checkpoint, read
+    # back and run: the stored codes and scales give the same output bits
+    from w8a8_int8_quantized_rmsnorm_b200 import checkpoint as ck
+    N = 512
+    x = workloads.activations(48, K, outlier_count=K // 100, seed=5).cuda()
+    lin = cr.ConvRotLinear(workloads.weight(N, K, seed=6).cuda(), weight_bits=bits, group=group)
+    y0 = lin(x)
+    p = str(tmp_path / "layer.safetensors")
+    ck.save_quantized_layers(p, {"model.layers.3.mlp.down_proj": lin.to_checkpoint()})
+    loaded = ck.load_quantized_layers(p)["model.layers.3.mlp.down_proj"]
+    assert loaded["meta"]["convrot_groupsize"] == group
+    lin2 = cr.ConvRotLinear.from_checkpoint(loaded)
+    y1 = lin2(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("sizes,K", [((4096, 1024, 1024), 4096), ((12288, 64), 4096), ((256, 48, 16), 512)])
+def test_fused_projection_set_equals_separate_linears(cr, sizes, K):
+    # one GEMM over concatenated rows gives each member's output bit for bit
+    M = 96
+    x = workloads.activations(M, K, outlier_count=K // 100, seed=7).cuda()
+    nw = workloads.norm_weight(K).cuda()
+    Ws = [workloads.weight(n, K, seed=10 + i).cuda() for i, n in enumerate(sizes)]
+    fused = cr.ConvRotFusedLinear(Ws, norm_w=nw, x_calib=x)
+    outs = fused(x)
+    for W, y in zip(Ws, outs):
+        lin = cr.ConvRotLinear(W, norm_w=fused.linear.norm_w, col_scale=fused.col_scale)
+        assert torch.equal(lin(x), y)
+    torch.cuda.synchronize()
+    assert cr.convrot_device_status() == 0

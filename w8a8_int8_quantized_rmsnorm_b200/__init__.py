@@ -22,7 +22,7 @@ __all__ = [
     "convrot_w4a8_linear", "convrot_int8_linear_noalloc", "convrot_int8_gemm_s32", "convrot_w4a8_gemm_s32",
     "convrot_swiglu_workspace_bytes", "convrot_int8_linear_swiglu", "convrot_w4a8_linear_swiglu",
     "convrot_interleave_gate_up", "convrot_fold_row_scales",
-    "Workspace", "ConvRotLinear", "ConvRotMLP",
+    "Workspace", "ConvRotLinear", "ConvRotFusedLinear", "ConvRotMLP",
 ]
 
 
@@ -323,6 +323,26 @@ class ConvRotLinear:
         self.workspace = Workspace(W.device.index)
 
     @classmethod
+    def from_checkpoint(cls, layer: dict, *, device=None, norm_w: Optional[torch.Tensor] = None,
+                        eps: float = 1e-6):
+        """A linear from an entry of checkpoint.load_quantized_layers (the stored
+        codes and row scales are used as they are; nothing is re-quantised)."""
+        self = cls.__new__(cls)
+        dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+        self.group, self.weight_bits, self.eps, self.norm_w = int(layer["group"]), int(layer["bits"]), eps, norm_w
+        self.Wq = torch.from_numpy(layer["Wq"]).to(dev)
+        self.s_row = torch.from_numpy(layer["s_row"]).to(dev)
+        self.N = self.Wq.shape[0]
+        self.K = self.Wq.shape[1] * (2 if self.weight_bits == 4 else 1)
+        self.workspace = Workspace(dev.index)
+        return self
+
+    def to_checkpoint(self) -> dict:
+        """The layer's stored form for checkpoint.save_quantized_layers."""
+        return {"Wq": self.Wq.cpu().numpy(), "s_row": self.s_row.cpu().numpy(),
+                "group": self.group, "bits": self.weight_bits}
+
+    @classmethod
     def with_smoothquant(cls, W, x_calib, norm_w, *, weight_bits=8, group=256, eps=1e-6, alpha=0.5):
         smooth, folded = convrot_smoothquant_calibrate(x_calib, norm_w, W, eps, alpha)
         return cls(W, weight_bits=weight_bits, group=group, norm_w=folded, col_scale=smooth, eps=eps)
@@ -332,6 +352,37 @@ class ConvRotLinear:
         if self.weight_bits == 8:
             return convrot_int8_linear(Xq, s_tok, self.Wq, self.s_row, out, self.workspace)
         return convrot_w4a8_linear(Xq, s_tok, self.Wq, self.s_row, out, self.workspace)
+
+    __call__ = forward
+
+
+class ConvRotFusedLinear:
+    """Several linears that read the same input, run as ONE GEMM over their
+    concatenated output rows: a fused projection set such as q/k/v of an
+    attention block, or a gated-DeltaNet input projection together with its
+    small-N companion (the MOSS-Image card quantises attention, gated-DeltaNet
+    projections and MLP linears).  Every row is quantised on its own, so the
+    fused layer's codes, scales and outputs are those of the separate layers;
+    one launch replaces several, and small-N members no longer under-fill the
+    GPU.  A shared SmoothQuant scale (with a norm) is calibrated over all
+    members' columns, since they share the input.
+    """
+
+    def __init__(self, weights, *, weight_bits: int = 8, group: int = 256,
+                 norm_w: Optional[torch.Tensor] = None, x_calib: Optional[torch.Tensor] = None,
+                 eps: float = 1e-6, alpha: float = 0.5):
+        W = torch.cat(list(weights))
+        self.sizes = [int(w.shape[0]) for w in weights]
+        col = None
+        if x_calib is not None and norm_w is not None:
+            col, norm_w = convrot_smoothquant_calibrate(x_calib, norm_w, W, eps, alpha)
+        self.col_scale = col
+        self.linear = ConvRotLinear(W, weight_bits=weight_bits, group=group, norm_w=norm_w,
+                                    col_scale=col, eps=eps)
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None):
+        """One output per member, as column views of the fused [M, sum N] result."""
+        return torch.split(self.linear(x, out), self.sizes, dim=1)
 
     __call__ = forward
 

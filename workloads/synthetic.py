@@ -155,6 +155,14 @@ WORKLOADS = {
     **{f"gate_up_m{m}": Workload(f"gate_up_m{m}", m, (Linear("gate_up", 24576, 4096),),
                                  outlier_frac=0.01, outlier_scale=20.0)
        for m in (1, 16, 128, 1024, 8192)},
+    # fused projection sets: q/k/v of the decoder layer as one GEMM behind the
+    # input RMSNorm (N = 4096 + 1024 + 1024), and a gated-DeltaNet-style input
+    # projection with its small-N companion (N = 12288 + 64; illustrative
+    # widths, the cards give none)
+    "attn_qkv_m2048": Workload("attn_qkv_m2048", 2048, (Linear("qkv_proj", 6144, 4096),),
+                               outlier_frac=0.005, outlier_scale=20.0, norm=True),
+    "gdn_in_proj_m2048": Workload("gdn_in_proj_m2048", 2048, (Linear("in_proj_qkvz_ba", 12352, 4096),),
+                                  outlier_frac=0.005, outlier_scale=20.0, norm=True),
     # the decoder layer's MLP block as one chain: RMSNorm + rotate-quantise,
     # gate/up GEMM with the SiLU(gate) * up epilogue, rotate-quantise of H,
     # down_proj; SmoothQuant folded into the norm and into up_proj's rows
