@@ -338,6 +338,33 @@ def smoothquant_scales(x, norm_w, eps: float, W, alpha: float = 0.5,
 
 
 # --------------------------------------------------------------------------
+# weight-only path: rotated activations kept in bf16, int8 weight codes
+# --------------------------------------------------------------------------
+def rotate_act(x, group: int = GROUP, norm_w=None, eps: float = 1e-6) -> np.ndarray:
+    """[RMSNorm] then the group rotation, without quantisation (float64).
+
+    The MOSS-Image card's "Matmul" row: the weight can also be dequantised for a
+    bf16 matmul.  A ConvRot weight is stored rotated (W' = W R), and
+    x W^T = (x R) W'^T, so the activation is rotated instead of the weight
+    being rotated back.
+    """
+    u = np.asarray(x, dtype=np.float64)
+    if norm_w is not None:
+        u = rmsnorm(u, norm_w, eps)
+    return rotate_groups(u, group)
+
+
+def weight_only_linear(Xr, Wq, s_row):
+    """y[m,n] = s_row[n] * sum_k Xr[m,k] Wq[n,k] (float64), and its bf16 rounding.
+
+    Xr is the rotated activation as the GEMM receives it (bf16 values);
+    returns (y_bf16, y64)."""
+    y = (np.asarray(Xr, dtype=np.float64) @ np.asarray(Wq, dtype=np.float64).T
+         * np.asarray(s_row, dtype=np.float64)[None, :])
+    return to_bf16(y), y
+
+
+# --------------------------------------------------------------------------
 # MLP boundary: gate/up linear with SiLU(gate) * up, and the down_proj fold
 # --------------------------------------------------------------------------
 SWIGLU_BLOCK = 16  # gate and up rows alternate in blocks of this many rows

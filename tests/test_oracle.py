@@ -492,3 +492,39 @@ def test_down_proj_fold_into_up_rows_preserves_the_mlp():
     q1, s1, _ = ref.quantize_weight(Wu / s[:, None])
     np.testing.assert_array_equal(q0, q1)
     np.testing.assert_allclose(ref.fold_smooth_into_rows(s0, s), s1, rtol=2e-7)
+
+
+# ---------------------------------------------------------------- weight-only path
+def test_weight_only_equals_the_plain_linear_for_a_representable_weight():
+    # W built from integer codes: W = (s * Wq) R, so the stored weight of W is
+    # exactly (Wq, s) and the weight-only path gives x W^T in float64
+    rng = np.random.default_rng(31)
+    N, K = 12, 512
+    Wq = rng.integers(-127, 128, (N, K)).astype(np.float64)
+    Wq[:, 0] = 127  # a full-range code in every row
+    s = rng.uniform(1e-3, 1e-2, N)
+    W = ref.rotate_groups(Wq * s[:, None])      # R is symmetric and orthogonal
+    q, s_row, _ = ref.quantize_weight(W)
+    np.testing.assert_array_equal(q, Wq)
+    x = rng.standard_normal((5, K))
+    _, y = ref.weight_only_linear(ref.rotate_act(x), q, s_row)
+    np.testing.assert_allclose(y, x @ W.T, rtol=1e-6, atol=1e-9)  # s_row is fp32
+
+
+def test_weight_only_one_hot_code_closed_form():
+    Xr = np.arange(12, dtype=np.float64).reshape(3, 4)
+    Wq = np.zeros((2, 4))
+    Wq[1, 2] = -3
+    _, y = ref.weight_only_linear(Xr, Wq, np.array([5.0, 0.5]))
+    np.testing.assert_array_equal(y, [[0, -3.0], [0, -9.0], [0, -15.0]])
+
+
+def test_rotate_act_is_the_rotation_of_the_norm():
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((3, 256))
+    w = rng.standard_normal(256) * 0.1
+    v = ref.rotate_act(x, 256, w, 1e-6)
+    # orthogonal rotation: row norms of the normalised input are kept
+    np.testing.assert_allclose(np.linalg.norm(v, axis=1), np.linalg.norm(ref.rmsnorm(x, w, 1e-6), axis=1),
+                               rtol=1e-13)
+    assert np.array_equal(ref.rotate_act(x, 0), x)
