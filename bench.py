@@ -250,7 +250,8 @@ def run_ours(args, rank, world, dev):
     w_sets = [[(l.Wq, l.s_row) for l in layers]] + \
              [[(l.Wq.clone(), l.s_row.clone()) for l in layers] for _ in range(copies - 1)]
     ws = cr.Workspace(dev.index)
-    Xq = [torch.empty(w.M, g["K"], dtype=torch.int8, device=dev) for g in groups]
+    wo = w.weight_only
+    Xq = [torch.empty(w.M, g["K"], dtype=torch.bfloat16 if wo else torch.int8, device=dev) for g in groups]
     st = [torch.empty(w.M, dtype=torch.float32, device=dev) for g in groups]
     Ys = [inputs[1] if l.swiglu else torch.empty(w.M, l.out_cols, dtype=torch.bfloat16, device=dev)
           for l in layers]
@@ -262,11 +263,17 @@ def run_ours(args, rank, world, dev):
     n_k2 = len(layers)
 
     def launch_k1(c, gi):
-        cr.convrot_rotate_quant_act(x_sets[c][gi], 256, norms[gi], 1e-6, out=(Xq[gi], st[gi]))
+        if wo:
+            cr.convrot_rotate_act_bf16(x_sets[c][gi], 256, norms[gi], 1e-6, out=Xq[gi])
+        else:
+            cr.convrot_rotate_quant_act(x_sets[c][gi], 256, norms[gi], 1e-6, out=(Xq[gi], st[gi]))
 
     def launch_k2(c, li):
         l = layers[li]
         Wq, s_row = w_sets[c][li]
+        if wo:
+            cr.convrot_weight_only_linear(Xq[l.group_in], Wq, s_row, out=Ys[li])
+            return
         (swiglu if l.swiglu else linear)(Xq[l.group_in], st[l.group_in], Wq, s_row, out=Ys[li],
                                          workspace=ws)
 
@@ -384,12 +391,17 @@ def run_ours(args, rank, world, dev):
     tokens = w.M * args.steps * world
     ops = w.ops() * args.steps * world
     secs = elapsed_ms / 1e3
-    k1_bytes = sum(w.M * g["K"] * 3 + 4 * w.M + (4 * g["K"] if norms[gi] is not None else 0)
-                   for gi, g in enumerate(groups))
-    k2_bytes = sum(w.M * l.lin.K + l.Wq.numel() + 2 * w.M * l.out_cols + 4 * (w.M + l.lin.N)
-                   for l in layers)
+    # algorithmic bytes: K1 reads bf16 and writes int8 codes + scales (bf16 on
+    # the weight-only path); K2 reads its activation (int8, or bf16 on the
+    # weight-only path), the weight, the scales and writes bf16
+    act_b = 2 if wo else 1
+    k1_bytes = sum(w.M * g["K"] * (2 + act_b) + (0 if wo else 4 * w.M) +
+                   (4 * g["K"] if norms[gi] is not None else 0) for gi, g in enumerate(groups))
+    k2_bytes = sum(act_b * w.M * l.lin.K + l.Wq.numel() + 2 * w.M * l.out_cols +
+                   (0 if wo else 4 * w.M) + 4 * l.lin.N for l in layers)
     k2_ops = w.ops()
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    # the weight-only GEMM multiplies in bf16: its tensor peak is the bf16 one
+    int8_peak = peaks["bf16_tflops"] * (1.0 if wo else INT8_PER_BF16)
     k2_achieved_tops = k2_ops / (statistics.mean(k2_ms) / 1e3) / 1e12
     k2_achieved_gbs = k2_bytes / (statistics.mean(k2_ms) / 1e3) / 1e9
     k1_achieved_gbs = k1_bytes / (statistics.mean(k1_ms) / 1e3) / 1e9
@@ -397,12 +409,15 @@ def run_ours(args, rank, world, dev):
     # ridge (~250 tokens) and weight-stream (HBM) bound below it
     ridge_bound = "tensor" if w.M > 256 else "hbm"
     if ridge_bound == "tensor":
-        roof = {"bound": "tensor", "kernel": "W8A8/W4A8 GEMM launch (tcgen05 kind::i8)",
+        roof = {"bound": "tensor", "kernel": ("weight-only GEMM launch (tcgen05 kind::f16, int8 weight codes)"
+                                              if wo else "W8A8/W4A8 GEMM launch (tcgen05 kind::i8)"),
                 "achieved": round(k2_achieved_tops, 1), "peak": round(int8_peak, 1),
                 "unit": "TOP/s", "frac": round(k2_achieved_tops / int8_peak, 4),
-                "peak_note": f"{peaks['source']}: 2 x dense bf16 burst {peaks['bf16_tflops']} TFLOP/s"}
+                "peak_note": (f"{peaks['source']}: dense bf16 burst {peaks['bf16_tflops']} TFLOP/s" if wo else
+                              f"{peaks['source']}: 2 x dense bf16 burst {peaks['bf16_tflops']} TFLOP/s")}
     else:
-        roof = {"bound": "hbm", "kernel": "W8A8/W4A8 GEMM launch (tcgen05 kind::i8)",
+        roof = {"bound": "hbm", "kernel": ("weight-only GEMM launch (tcgen05 kind::f16, int8 weight codes)"
+                                           if wo else "W8A8/W4A8 GEMM launch (tcgen05 kind::i8)"),
                 "achieved": round(k2_achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(k2_achieved_gbs / peaks["hbm_gbs"], 4),
                 "peak_note": f"{peaks['source']} copy bandwidth"}
@@ -420,13 +435,14 @@ def run_ours(args, rank, world, dev):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "i8",
+        "dtype": "bf16" if wo else "i8",
         "data": "synthetic (seeded; no trained weights or datasets)",
         "tops": round(ops / secs / 1e12, 1),
         "config": {
             "workload": args.workload, "M": w.M,
             "linears": [[l.name, l.N, l.K] for l in w.linears], "layers": w.layers,
             "weight_bits": w.weight_bits, "group": 256, "rmsnorm": w.norm,
+            **({"path": "weight-only: rotated bf16 activations x int8 weight codes (bf16 MMA)"} if wo else {}),
             **({"block": "down(SiLU(gate(x)) * up(x)); gate/up as one GEMM with the SwiGLU epilogue"}
                if w.mlp else {}),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -486,6 +502,13 @@ def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
         host_x = [x.cpu().pin_memory() for x in inputs]
         host_y = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16).pin_memory() for l in layers]
         step = None
+        if w.weight_only:
+            def step():
+                xs = [h.to(dev, non_blocking=True) for h in host_x]
+                xr = [cr.convrot_rotate_act_bf16(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
+                for li, l in enumerate(layers):
+                    host_y[li].copy_(cr.convrot_weight_only_linear(xr[l.group_in], l.Wq, l.s_row),
+                                     non_blocking=True)
 
     def layer_step():
         xs = [h.to(dev, non_blocking=True) for h in host_x]
@@ -543,6 +566,13 @@ def oracle_step_runner(w, sample_tokens):
             else:
                 o = ref.quantize_weight_w4(W, 256, col)
                 preps.append((gi, None, o["s_row"], o["packed"]))
+
+    if w.weight_only:
+        def run_wo():
+            acts = [ref.to_bf16(ref.rotate_act(xs[g], 256, nws[g], 1e-6)) for g in range(len(groups))]
+            for gi, Wq, s_row, _ in preps:
+                ref.weight_only_linear(acts[gi], Wq, s_row)
+        return run_wo
 
     def run():
         acts = [ref.rotate_quant_act(xs[g], 256, nws[g], 1e-6) for g in range(len(groups))]

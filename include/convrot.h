@@ -271,6 +271,30 @@ convrot_status convrot_fold_row_scales(float* s_row, const float* smooth, int n,
                                        convrot_stream_t stream);
 
 /*
+ * Weight-only path ("Matmul" row of the MOSS-Image card's file table: the
+ * weight can also be dequantised for a bf16 matmul).  The stored weight is
+ * ConvRot-rotated, so instead of rotating the weight back the activation is
+ * rotated by the same Hadamard and kept in bf16 (no activation quantisation):
+ *   Xr[m,k] = bf16_rn(r * (x * (1 + norm_w)) * R)      convrot_rotate_act_bf16
+ *             (norm_w NULL: no RMSNorm, r = 1; group 256, 16 or 0)
+ *   Y[m,n]  = bf16_rn(s_row[n] * sum_k Xr[m,k] * Wq[n,k])   convrot_weight_only_linear
+ * The int8 codes are expanded to bf16 (exactly) in shared memory and
+ * multiplied on the tensor cores (bf16 inputs, fp32 accumulation), so Y
+ * approximates x W^T with the weight's int8 rounding only.
+ * x bf16 [M, K], Xr bf16 [M, K], Wq int8 [N, K], s_row fp32 [N], Y bf16 [M, N];
+ * K % 16 == 0, N % 8 == 0; all 16-byte aligned.  No workspace is needed.
+ * convrot_weight_only_gemm_f32 writes the raw fp32 accumulators instead
+ * (acc fp32 [M, N]) for accuracy checks.
+ */
+convrot_status convrot_rotate_act_bf16(const void* x, int M, int K, int group,
+                                       const float* norm_w, float eps, void* Xr,
+                                       convrot_stream_t stream);
+convrot_status convrot_weight_only_linear(const void* Xr, const int8_t* Wq, const float* s_row,
+                                          int M, int N, int K, void* Y, convrot_stream_t stream);
+convrot_status convrot_weight_only_gemm_f32(const void* Xr, const int8_t* Wq, int M, int N, int K,
+                                            float* acc, convrot_stream_t stream);
+
+/*
  * Allocation-free W8A8 linear.  The model cards have no counterpart: this is
  * an interface addition for callers that cannot allocate device memory where
  * they run the layer (plugins without an allocator, runtimes whose device

@@ -22,6 +22,7 @@ __all__ = [
     "convrot_w4a8_linear", "convrot_int8_linear_noalloc", "convrot_int8_gemm_s32", "convrot_w4a8_gemm_s32",
     "convrot_swiglu_workspace_bytes", "convrot_int8_linear_swiglu", "convrot_w4a8_linear_swiglu",
     "convrot_interleave_gate_up", "convrot_fold_row_scales",
+    "convrot_rotate_act_bf16", "convrot_weight_only_linear", "convrot_weight_only_gemm_f32",
     "Workspace", "ConvRotLinear", "ConvRotFusedLinear", "ConvRotMLP",
 ]
 
@@ -243,6 +244,46 @@ def convrot_w4a8_gemm_s32(Xq, Wq4, workspace: Optional[Workspace] = None):
     return acc
 
 
+# ---------------------------------------------------------------- weight-only path
+def convrot_rotate_act_bf16(x: torch.Tensor, group: int = 256, norm_w: Optional[torch.Tensor] = None,
+                            eps: float = 1e-6, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Xr = bf16([RMSNorm] x rotated by the group Hadamard), not quantised."""
+    _need(x, torch.bfloat16, "x", 2)
+    if norm_w is not None:
+        _need(norm_w, torch.float32, "norm_w", 1)
+    M, K = x.shape
+    Xr = torch.empty(M, K, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check("convrot_rotate_act_bf16", lib().convrot_rotate_act_bf16(
+        _ptr(x), M, K, group, _ptr(norm_w), eps, _ptr(Xr), _stream(x.device)))
+    return Xr
+
+
+def _wo_check(Xr, Wq):
+    _need(Xr, torch.bfloat16, "Xr", 2)
+    _need(Wq, torch.int8, "Wq", 2)
+    if Xr.shape[1] != Wq.shape[1]:
+        raise ValueError("weight and activation disagree on K")
+    return Xr.shape[0], Wq.shape[0], Xr.shape[1]
+
+
+def convrot_weight_only_linear(Xr, Wq, s_row, out=None):
+    """Y = bf16(s_row * (Xr @ Wq^T)) on rotated bf16 activations, int8 weights."""
+    M, N, K = _wo_check(Xr, Wq)
+    _need(s_row, torch.float32, "s_row", 1)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xr.device) if out is None else out
+    _check("convrot_weight_only_linear", lib().convrot_weight_only_linear(
+        _ptr(Xr), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), _stream(Xr.device)))
+    return Y
+
+
+def convrot_weight_only_gemm_f32(Xr, Wq):
+    M, N, K = _wo_check(Xr, Wq)
+    acc = torch.empty(M, N, dtype=torch.float32, device=Xr.device)
+    _check("convrot_weight_only_gemm_f32", lib().convrot_weight_only_gemm_f32(
+        _ptr(Xr), _ptr(Wq), M, N, K, _ptr(acc), _stream(Xr.device)))
+    return acc
+
+
 # ---------------------------------------------------------------- MLP boundary
 def convrot_swiglu_workspace_bytes(M: int, I: int, K: int, weight_bits: int = 8) -> int:
     return int(lib().convrot_swiglu_workspace_bytes(M, I, K, weight_bits))
@@ -346,6 +387,14 @@ class ConvRotLinear:
     def with_smoothquant(cls, W, x_calib, norm_w, *, weight_bits=8, group=256, eps=1e-6, alpha=0.5):
         smooth, folded = convrot_smoothquant_calibrate(x_calib, norm_w, W, eps, alpha)
         return cls(W, weight_bits=weight_bits, group=group, norm_w=folded, col_scale=smooth, eps=eps)
+
+    def forward_weight_only(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """The same layer with bf16 activations: rotate (no quantisation), then the
+        bf16 tensor-core GEMM over the int8 weight codes (int8 weights only)."""
+        if self.weight_bits != 8:
+            raise ValueError("the weight-only path takes int8 weights")
+        Xr = convrot_rotate_act_bf16(x, self.group, self.norm_w, self.eps)
+        return convrot_weight_only_linear(Xr, self.Wq, self.s_row, out)
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         Xq, s_tok = convrot_rotate_quant_act(x, self.group, self.norm_w, self.eps)

@@ -302,10 +302,14 @@ int pick_bn_swap(int M) {
 // kernel, CTA pairs (clusters of two) for the pair kernel.
 // `clusters4` is the number of co-resident four-CTA clusters of the split
 // pair kernel (0 if unavailable).
-GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int clusters4) {
+// wbf: the weight-only path (bf16 activations, int8 weights expanded to bf16,
+// fp32 accumulators): single-CTA tiles, 64 K elements per stage, plain waves
+// only (its fp32 partial sums have no split-tile reduction).
+GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int clusters4,
+                   bool wbf = false) {
   GemmPlan p{};
   p.swap = M <= 128;
-  p.pair = !p.swap && pairs > 0;
+  p.pair = !p.swap && pairs > 0 && !wbf;
   p.bn = p.swap ? pick_bn_swap(M) : 256;
   const int rowsA = p.swap ? N : M;
   const int rowsB = p.swap ? M : N;
@@ -313,12 +317,12 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   p.tilesA = (rowsA + tileA - 1) / tileA;
   p.tilesB = (rowsB + p.bn - 1) / p.bn;
   p.num_tiles = p.tilesA * p.tilesB;
-  const int stage_k = GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
+  const int stage_k = wbf ? GEMM_BK / 2 : GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
   p.num_kb = (K + stage_k - 1) / stage_k;
   // One wave of 256 x 256 tiles that fits the co-resident clusters: each tile
   // is split in two K halves over two CTA pairs whose partial sums meet in
   // shared memory (no stream-K workspace, no L2 round trip).
-  if (p.pair && !w4 && clusters4 > 0 && p.num_kb >= 2 && p.num_tiles <= clusters4) {
+  if (p.pair && !w4 && !wbf && clusters4 > 0 && p.num_kb >= 2 && p.num_tiles <= clusters4) {
     p.split = true;
     p.grid = p.num_tiles;
     p.dp_tiles = 0;
@@ -343,7 +347,7 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   const long long sk_total = static_cast<long long>(sk_tiles) * p.num_kb;
   const long long t_sk = static_cast<long long>(p.dp_tiles / p.grid) * p.num_kb +
                          (sk_total + p.grid - 1) / p.grid + fixup_stages(p.swap, p.bn);
-  if (t_dp <= t_sk) {
+  if (wbf || t_dp <= t_sk) {
     p.dp_tiles = p.num_tiles;
     sk_tiles = 0;
   }
@@ -472,11 +476,11 @@ size_t ws_bytes(const GemmPlan& p) {
   return kCounterBytes + p.ws_slot_bytes;
 }
 
-template <int BN, bool SWAP, bool W4, int EPI>
+template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
 convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
                              GemmArgs a, int grid, cudaStream_t st) {
-  using SM = GemmSmem<BN, W4, SWAP>;
-  auto k = gemm_kernel<BN, SWAP, W4, EPI>;
+  using SM = GemmSmem<BN, W4 || WBF, SWAP>;
+  auto k = gemm_kernel<BN, SWAP, W4, EPI, WBF>;
   // as many stages as fit next to the epilogue staging and the barriers in
   // 227 KB; at least ~116 KB so that a second CTA never shares the SM's TMEM
   const int avail = 227 * 1024 - 1024 - SM::total(0);
@@ -492,8 +496,68 @@ convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const
       return CONVROT_ERR_CUDA;
     configured_device_mask |= bit;
   }
-  constexpr int threads = W4 ? 320 : 192;
+  constexpr int threads = (W4 || WBF) ? 320 : 192;
   return launch_pdl(k, dim3(grid), dim3(threads), smem, st, 1, ma, mb, my, a);
+}
+
+template <int EPI>
+convrot_status launch_wbf(bool swap, int bn, const CUtensorMap& ma, const CUtensorMap& mb,
+                          const CUtensorMap& my, const GemmArgs& a, int grid, cudaStream_t st) {
+  if (!swap) return launch_gemm_t<256, false, false, EPI, true>(ma, mb, my, a, grid, st);
+  switch (bn) {
+    case 16: return launch_gemm_t<16, true, false, EPI, true>(ma, mb, my, a, grid, st);
+    case 32: return launch_gemm_t<32, true, false, EPI, true>(ma, mb, my, a, grid, st);
+    case 64: return launch_gemm_t<64, true, false, EPI, true>(ma, mb, my, a, grid, st);
+    default: return launch_gemm_t<128, true, false, EPI, true>(ma, mb, my, a, grid, st);
+  }
+}
+
+// Weight-only path: Xr bf16 [M, K] (rotated activations), Wq int8 [N, K];
+// out bf16 Y = (Xr Wq^T) * s_row, or raw fp32 accumulators (f32_out).
+convrot_status run_gemm_wbf(const void* Xr, const int8_t* Wq, const float* s_row, int M, int N,
+                            int K, void* out, bool f32_out, cudaStream_t st) {
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
+  const GemmPlan p = plan_gemm(M, N, K, d.sms, 0, false, 0, true);
+  const int bn = p.bn;
+  CUtensorMap mx, mw, my;
+  std::memset(&my, 0, sizeof(my));
+  // K atoms of 64 elements: 128 bytes of a bf16 row (swizzled like the int8
+  // atoms), 64 bytes of an int8 weight row (expanded in shared memory)
+  const uint32_t x_box_rows = p.swap ? bn : GEMM_BM;
+  const uint32_t w_box_rows = p.swap ? GEMM_BM : bn;
+  if (!make_map(&mx, Xr, M, K, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_box_rows, GEMM_BK / 2, true))
+    return CONVROT_ERR_CUDA;
+  if (!make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK / 2, false)) return CONVROT_ERR_CUDA;
+  bool ok;
+  if (!p.swap) {
+    ok = f32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32, true)
+                 : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, 64, true);
+  } else {
+    const uint32_t cw = bn < 32 ? bn : 32;
+    ok = f32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cw, 128, false)
+                 : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cw, 128, false);
+  }
+  if (!ok) return CONVROT_ERR_CUDA;
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.rowsA = p.swap ? N : M;
+  a.rowsB = p.swap ? M : N;
+  a.tilesA = p.tilesA;
+  a.tilesB = p.tilesB;
+  a.num_tiles = p.num_tiles;
+  a.num_kb = p.num_kb;
+  a.dp_tiles = p.dp_tiles;
+  a.s_tok = nullptr;
+  a.s_row = s_row;
+  a.srow_vec = (s_row != nullptr && aligned(s_row, 16)) ? 1 : 0;
+  a.out = out;
+  const CUtensorMap& ma = p.swap ? mw : mx;
+  const CUtensorMap& mb = p.swap ? mx : mw;
+  return f32_out ? launch_wbf<EPI_S32>(p.swap, bn, ma, mb, my, a, p.grid, st)
+                 : launch_wbf<EPI_BF16>(p.swap, bn, ma, mb, my, a, p.grid, st);
 }
 
 template <bool SWAP, bool W4, int EPI>
@@ -837,6 +901,50 @@ convrot_status convrot_w4a8_linear_swiglu(const int8_t* Xq, const float* s_tok,
                                           size_t workspace_bytes, convrot_stream_t stream) {
   return swiglu_common(Xq, s_tok, Wq4_gu, true, s_row_gu, M, I, K, H, workspace,
                        workspace_bytes, stream);
+}
+
+convrot_status convrot_rotate_act_bf16(const void* x, int M, int K, int group,
+                                       const float* norm_w, float eps, void* Xr,
+                                       convrot_stream_t stream) {
+  if (M < 0) return CONVROT_ERR_SHAPE;
+  const convrot_status g = check_group(group, K, 16);
+  if (g != CONVROT_OK) return g;
+  if (norm_w && !(eps >= 0.f)) return CONVROT_ERR_SHAPE;
+  if (M == 0) return CONVROT_OK;
+  if (!x || !Xr) return CONVROT_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(Xr, 16)) return CONVROT_ERR_ALIGN;
+  if (norm_w && !aligned(norm_w, 16)) return CONVROT_ERR_ALIGN;
+  RowQuantArgs a{};
+  a.src = static_cast<const uint16_t*>(x);
+  a.vec = norm_w;
+  a.dstb = static_cast<uint16_t*>(Xr);
+  a.rows = M;
+  a.K = K;
+  a.eps = eps;
+  return norm_w ? launch_rowquant_pre<PRE_NORM, QK_BF16>(a, group, as_cuda(stream))
+                : launch_rowquant_pre<PRE_NONE, QK_BF16>(a, group, as_cuda(stream));
+}
+
+static convrot_status weight_only_common(const void* Xr, const int8_t* Wq, const float* s_row,
+                                         int M, int N, int K, void* out, bool f32_out,
+                                         convrot_stream_t stream) {
+  const convrot_status sh = check_gemm_shape(M, N, K, false);
+  if (sh != CONVROT_OK) return sh;
+  if (M == 0 || N == 0) return CONVROT_OK;
+  if (!Xr || !Wq || !out || (!f32_out && !s_row)) return CONVROT_ERR_NULL;
+  if (!aligned(Xr, 16) || !aligned(Wq, 16) || !aligned(out, 16) || (s_row && !aligned(s_row, 4)))
+    return CONVROT_ERR_ALIGN;
+  return run_gemm_wbf(Xr, Wq, s_row, M, N, K, out, f32_out, as_cuda(stream));
+}
+
+convrot_status convrot_weight_only_linear(const void* Xr, const int8_t* Wq, const float* s_row,
+                                          int M, int N, int K, void* Y, convrot_stream_t stream) {
+  return weight_only_common(Xr, Wq, s_row, M, N, K, Y, false, stream);
+}
+
+convrot_status convrot_weight_only_gemm_f32(const void* Xr, const int8_t* Wq, int M, int N, int K,
+                                            float* acc, convrot_stream_t stream) {
+  return weight_only_common(Xr, Wq, nullptr, M, N, K, acc, true, stream);
 }
 
 convrot_status convrot_interleave_gate_up(const void* Wg, const void* Wu, int I,

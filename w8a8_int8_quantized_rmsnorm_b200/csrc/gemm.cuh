@@ -209,17 +209,32 @@ struct GemmSmem {
   }
 };
 
+// Accumulator value: int32 for the integer MMAs, fp32 bits for kind::f16.
+template <bool F32ACC>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+  return F32ACC ? __uint_as_float(r) : static_cast<float>(static_cast<int32_t>(r));
+}
+
 // One CTA per SM.  Registers are allocated per SM sub-partition (16K each, a
 // CTA's warps spread over four): with 6 (10) warps, two (three) share one, so
 // 255 (168) registers per thread is the most a launch can use.
-template <int BN, bool SWAP, bool W4, int EPI>
-__global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
+//
+// WBF (weight-only path): the activation operand is bf16 (already rotated),
+// the int8 weight tile is expanded to bf16 in shared memory by the converter
+// warps (the int4 path's staging: 64 bytes per row in, 128 bytes out, one
+// K atom = 64 elements per stage), the MMA is kind::f16 with an fp32
+// accumulator and the epilogue scales by s_row only.
+template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
+__global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WBF) ? 168 : 255)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, GemmArgs a) {
-  using SM = GemmSmem<BN, W4, SWAP>;
+  constexpr bool CONV = W4 || WBF;  // a converter stage between TMA and the MMA
+  static_assert(!(W4 && WBF), "int4 weights have no weight-only path");
+  static_assert(!(WBF && EPI == EPI_SWIGLU), "the weight-only path has no SwiGLU epilogue");
+  using SM = GemmSmem<BN, CONV, SWAP>;
   constexpr int CW = SM::CW;
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
-  constexpr uint32_t IDESC = idesc_s8s8s32(GEMM_BM, BN);
+  constexpr uint32_t IDESC = WBF ? idesc_bf16_f32(GEMM_BM, BN) : idesc_s8s8s32(GEMM_BM, BN);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -278,7 +293,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
       const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_last();
       const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_first();
       uint32_t tx = 0;
-      if (W4) {
+      if (CONV) {
         tx = SWAP ? (SM::P_BYTES + SM::B_BYTES) : (SM::A_BYTES + SM::P_BYTES);
       } else {
         tx = SM::A_BYTES + SM::B_BYTES;
@@ -289,18 +304,15 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
       // that tiles first touched in DRAM are in L2 when their load is issued
       constexpr int KA = SM::KA;
       const int pfd = S + GEMM_PREFETCH_ATOMS / KA;
+      // innermost TMA coordinate of K atom `atom`: int8 bytes, or half of that
+      // for packed int4 weights; WBF atoms are 64 elements of either operand
+      auto xa = [](int atom) { return (W4 && SWAP) || WBF ? atom * (GEMM_BK / 2) : atom * GEMM_BK; };
+      auto xb = [](int atom) { return (W4 && !SWAP) || WBF ? atom * (GEMM_BK / 2) : atom * GEMM_BK; };
       auto prefetch = [&](int ta, int tb, int kb) {
 #pragma unroll
         for (int j = 0; j < KA; ++j) {
-          const int k0 = (kb * KA + j) * GEMM_BK;
-          if (W4 && SWAP)
-            tma_prefetch_l2_2d(&tmA, k0 / 2, ta * GEMM_BM);
-          else
-            tma_prefetch_l2_2d(&tmA, k0, ta * GEMM_BM);
-          if (W4 && !SWAP)
-            tma_prefetch_l2_2d(&tmB, k0 / 2, tb * BN);
-          else
-            tma_prefetch_l2_2d(&tmB, k0, tb * BN);
+          tma_prefetch_l2_2d(&tmA, xa(kb * KA + j), ta * GEMM_BM);
+          tma_prefetch_l2_2d(&tmB, xb(kb * KA + j), tb * BN);
         }
       };
       while (ok && sched.next(seg)) {
@@ -320,16 +332,16 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
 #pragma unroll
           for (int j = 0; j < KA; ++j) {
             // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
-            const int k0 = (kb * KA + j) * GEMM_BK;
-            if (W4 && SWAP)
-              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmA, &full[s], k0 / 2, ta * GEMM_BM,
+            const int atom = kb * KA + j;
+            if (CONV && SWAP)
+              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmA, &full[s], xa(atom), ta * GEMM_BM,
                           pol_a);
             else
-              tma_load_2d(st + j * SM::A_ATOM, &tmA, &full[s], k0, ta * GEMM_BM, pol_a);
-            if (W4 && !SWAP)
-              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], k0 / 2, tb * BN, pol_b);
+              tma_load_2d(st + j * SM::A_ATOM, &tmA, &full[s], xa(atom), ta * GEMM_BM, pol_a);
+            if (CONV && !SWAP)
+              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], xb(atom), tb * BN, pol_b);
             else
-              tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, &full[s], k0, tb * BN, pol_b);
+              tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, &full[s], xb(atom), tb * BN, pol_b);
           }
           if (kb + pfd < seg.kb1) prefetch(ta, tb, kb + pfd);
           if (kb == win)
@@ -359,7 +371,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
-          if (!mbar_wait(W4 ? &conv[s] : &full[s], ph, abort_flag, SITE_MMA_FULL)) {
+          if (!mbar_wait(CONV ? &conv[s] : &full[s], ph, abort_flag, SITE_MMA_FULL)) {
             ok = false;
             break;
           }
@@ -370,9 +382,13 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
           for (int j = 0; j < SM::KA; ++j) {
 #pragma unroll
             for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
-              mma_s8(d, sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K),
-                     sw128_kmajor_desc(sb + j * SM::B_ATOM + k * GEMM_UMMA_K), IDESC,
-                     (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u);
+              const uint64_t ad = sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K);
+              const uint64_t bd = sw128_kmajor_desc(sb + j * SM::B_ATOM + k * GEMM_UMMA_K);
+              const uint32_t acc = (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u;
+              if (WBF)
+                mma_bf16(d, ad, bd, IDESC, acc);
+              else
+                mma_s8(d, ad, bd, IDESC, acc);
             }
           }
           mma_commit(&empty[s]);
@@ -478,7 +494,7 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
           const int m = arow;
           const int m0 = ta * GEMM_BM + 32 * q;
           float st = 0.f;
-          if (EPI != EPI_S32 && m < a.M) st = a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
+          if (EPI != EPI_S32 && m < a.M) st = WBF ? 1.0f : a.s_tok[m] * (W4 ? 0.0625f : 1.0f);
 #pragma unroll 1
           for (int oc = 0; oc < (EPI == EPI_SWIGLU ? BN / 128 : 0); ++oc) {
             // MLP boundary: 128 accumulator columns (four blocks of 16 gate and
@@ -590,8 +606,8 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
                 uint32_t w[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                  const float y0 = static_cast<float>(static_cast<int32_t>(rr[jb + 2 * h])) * st * sr[2 * h];
-                  const float y1 = static_cast<float>(static_cast<int32_t>(rr[jb + 2 * h + 1])) * st * sr[2 * h + 1];
+                  const float y0 = acc_value<WBF>(rr[jb + 2 * h]) * st * sr[2 * h];
+                  const float y1 = acc_value<WBF>(rr[jb + 2 * h + 1]) * st * sr[2 * h + 1];
                   w[h] = pack_bf16x2(y0, y1);
                 }
                 st_shared_v4(buf + lane * 128 + ((c16 ^ sw) << 4), w[0], w[1], w[2], w[3]);
@@ -682,8 +698,8 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
               uint8_t* dst = xb + j * (128 * ES) + nl * ES;
               if (EPI == EPI_BF16) {
                 const int m = m0 + j;
-                const float st = m < a.M ? __ldg(a.s_tok + m) : 0.f;
-                const float v = static_cast<float>(static_cast<int32_t>(r[j])) * st * sr;
+                const float st = m < a.M ? (WBF ? 1.0f : __ldg(a.s_tok + m)) : 0.f;
+                const float v = acc_value<WBF>(r[j]) * st * sr;
                 const __nv_bfloat16 hb = __float2bfloat16_rn(v);
                 asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_addr(dst)),
                              "h"(*reinterpret_cast<const unsigned short*>(&hb))
@@ -720,8 +736,9 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
     // the staged outputs must have been read before the CTA exits; the global
     // writes themselves complete before the grid does
     if (lane == 0) bulk_wait_group_read<0>();
-  } else if (W4) {
-    // ------------------------------------------------------------ int4 unpack
+  } else if (CONV) {
+    // ------------------------------------------------------------ int4 unpack /
+    // int8 -> bf16 (WBF)
     const int ct = threadIdx.x - 192;  // 0..127
     constexpr int WR = SM::W_ROWS;
     uint32_t it = 0;
@@ -744,10 +761,28 @@ __global__ void __launch_bounds__(W4 ? 320 : 192) __maxnreg__(W4 ? 168 : 255)
           uint32_t o[8];
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            const uint32_t lo = (w[h] << 4) & 0xF0F0F0F0u;
-            const uint32_t hi = w[h] & 0xF0F0F0F0u;
-            o[2 * h] = __byte_perm(lo, hi, 0x5140);
-            o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+            if (WBF) {
+              // four int8 codes q -> four bf16, exactly, on the full-rate ALU:
+              // u = q + 128 (the sign bit flipped) goes into the low byte of
+              // the fp32 2^23 + u, and subtracting 2^23 + 128 leaves q; q has
+              // at most 8 significant bits, so its bf16 is the upper half
+              const uint32_t u = w[h] ^ 0x80808080u;
+              const uint64_t m01 = static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7540)) |
+                                   (static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7541)) << 32);
+              const uint64_t m23 = static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7542)) |
+                                   (static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7543)) << 32);
+              const uint64_t bias = 0x4B0000804B000080ull;  // (2^23 + 128, 2^23 + 128)
+              uint64_t f01, f23;
+              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f01) : "l"(m01), "l"(bias));
+              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f23) : "l"(m23), "l"(bias));
+              o[2 * h] = __byte_perm(static_cast<uint32_t>(f01), static_cast<uint32_t>(f01 >> 32), 0x7632);
+              o[2 * h + 1] = __byte_perm(static_cast<uint32_t>(f23), static_cast<uint32_t>(f23 >> 32), 0x7632);
+            } else {
+              const uint32_t lo = (w[h] << 4) & 0xF0F0F0F0u;
+              const uint32_t hi = w[h] & 0xF0F0F0F0u;
+              o[2 * h] = __byte_perm(lo, hi, 0x5140);
+              o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+            }
           }
           const int sw = r & 7;
           *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);

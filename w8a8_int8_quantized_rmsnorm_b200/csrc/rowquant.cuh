@@ -31,13 +31,16 @@
 namespace convrot {
 
 enum PreOp { PRE_NONE = 0, PRE_NORM = 1, PRE_COLSCALE = 2 };
-enum QuantKind { QK_INT8 = 0, QK_INT4 = 1 };
+// QK_BF16: no quantisation; the rotated (and normalised) row is stored in
+// bf16 for the weight-only path
+enum QuantKind { QK_INT8 = 0, QK_INT4 = 1, QK_BF16 = 2 };
 
 struct RowQuantArgs {
   const uint16_t* src;  // [rows, K] bf16 bits
   const float* vec;     // [K]: RMSNorm weight w (PRE_NORM) or column scale (PRE_COLSCALE)
   int8_t* dst8;         // [rows, K]      (QK_INT8)
   uint8_t* dst4;        // [rows, K / 2]  (QK_INT4)
+  uint16_t* dstb;       // [rows, K] bf16 (QK_BF16)
   float* scale;         // [rows]
   int rows;
   int K;
@@ -263,6 +266,30 @@ __device__ __forceinline__ void rq_store_int8(const RowQuantArgs& a, int8_t* row
   }
 }
 
+// The rotated values times `scale`, rounded once to bf16 (register j of the
+// 32h + 16q block holds element g*256 + 128h + 32L + 16q + (j mod 16)).
+__device__ __forceinline__ void rq_store_bf16(const RowQuantArgs& a, uint16_t* row, int g, int L,
+                                              bool ok, const float (&v)[64], float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int j = 32 * h + 16 * q + 2 * k;
+        const __nv_bfloat162 b = __floats2bfloat162_rn(v[j] * scale, v[j + 1] * scale);
+        w[k] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      const int e = g * 256 + 128 * h + 32 * L + 16 * q;
+      if (ok && e < a.K) {
+        st_v4(row + e, make_uint4(w[0], w[1], w[2], w[3]));
+        st_v4(row + e + 8, make_uint4(w[4], w[5], w[6], w[7]));
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ float rq_sse_int4(const float (&v)[64], float s) {
   float e0 = 0.f, e1 = 0.f;
 #pragma unroll
@@ -363,7 +390,22 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
       rowfac *= 1.0 / sqrt(ms + static_cast<double>(a.eps));
     }
 
-    if (QK == QK_INT8) {
+    if (QK == QK_BF16) {
+      const float scale = static_cast<float>(rowfac);
+      uint16_t* dst_row = a.dstb + static_cast<size_t>(row_ok ? row : 0) * a.K;
+      if (RESIDENT) {
+        const int g = t >> 2;
+        rq_store_bf16(a, dst_row, g, L, row_ok && g < G, v, scale);
+      } else {
+        for (int p = 0; p < a.passes; ++p) {
+          const int g = (t + p * a.team) >> 2;
+          float sq2 = 0.f;
+          rq_load<PRE>(a, src_row, g, L, row_ok && g < G, v, sq2);
+          rq_transform<GRP>(v, lane);
+          rq_store_bf16(a, dst_row, g, L, row_ok && g < G, v, scale);
+        }
+      }
+    } else if (QK == QK_INT8) {
       const float inv = amax > 0.f ? 127.0f / amax : 0.0f;
       if (row_ok && t == 0)
         a.scale[row] = amax > 0.f ? static_cast<float>(static_cast<double>(amax) * rowfac / 127.0) : 0.0f;

@@ -115,6 +115,9 @@ class Workload:
     # projection (N = 2 I rows, gate and up interleaved), linears[1] down_proj,
     # whose input is the block's intermediate H instead of fresh activations
     mlp: bool = False
+    # weight-only path: rotated bf16 activations (no quantisation) and the bf16
+    # tensor-core GEMM over the int8 weight codes
+    weight_only: bool = False
 
     def n_outliers(self, K: int) -> int:
         if self.outlier_count:
@@ -163,6 +166,12 @@ WORKLOADS = {
                                outlier_frac=0.005, outlier_scale=20.0, norm=True),
     "gdn_in_proj_m2048": Workload("gdn_in_proj_m2048", 2048, (Linear("in_proj_qkvz_ba", 12352, 4096),),
                                   outlier_frac=0.005, outlier_scale=20.0, norm=True),
+    # weight-only path on the fused gate/up shape: decode (weight-stream bound,
+    # int8 weights are half the bytes of bf16) and prefill (bf16 tensor rate)
+    **{f"weight_only_gate_up_m{m}": Workload(f"weight_only_gate_up_m{m}", m,
+                                             (Linear("gate_up", 24576, 4096),),
+                                             outlier_frac=0.01, outlier_scale=20.0, weight_only=True)
+       for m in (16, 2048)},
     # the decoder layer's MLP block as one chain: RMSNorm + rotate-quantise,
     # gate/up GEMM with the SiLU(gate) * up epilogue, rotate-quantise of H,
     # down_proj; SmoothQuant folded into the norm and into up_proj's rows
