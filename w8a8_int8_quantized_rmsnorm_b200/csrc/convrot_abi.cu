@@ -317,7 +317,8 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   p.tilesA = (rowsA + tileA - 1) / tileA;
   p.tilesB = (rowsB + p.bn - 1) / p.bn;
   p.num_tiles = p.tilesA * p.tilesB;
-  const int stage_k = wbf ? GEMM_BK / 2 : GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
+  const int stage_k = wbf ? (GEMM_BK / 2) * wbf_katoms(p.swap, p.bn)
+                          : GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
   p.num_kb = (K + stage_k - 1) / stage_k;
   // One wave of 256 x 256 tiles that fits the co-resident clusters: each tile
   // is split in two K halves over two CTA pairs whose partial sums meet in
@@ -479,7 +480,7 @@ size_t ws_bytes(const GemmPlan& p) {
 template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
 convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
                              GemmArgs a, int grid, cudaStream_t st) {
-  using SM = GemmSmem<BN, W4 || WBF, SWAP>;
+  using SM = GemmSmem<BN, W4 || WBF, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0>;
   auto k = gemm_kernel<BN, SWAP, W4, EPI, WBF>;
   // as many stages as fit next to the epilogue staging and the barriers in
   // 227 KB; at least ~116 KB so that a second CTA never shares the SM's TMEM

@@ -61,6 +61,10 @@ constexpr int GEMM_PREFETCH_ATOMS = 8;  // L2 prefetch this many K atoms beyond 
 __host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
   return w4 ? (pair ? 2 : 1) : ((pair || swap) ? 2 : 1);
 }
+
+// K atoms per stage of the weight-only path: two for the small token tiles of
+// the swapped roles (a stage then stays near 52 KB), one otherwise.
+__host__ __device__ constexpr int wbf_katoms(bool swap, int bn) { return (swap && bn <= 64) ? 2 : 1; }
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
 // SiLU(gate) * up of the MLP boundary: the weight rows alternate in blocks of
@@ -183,17 +187,19 @@ __device__ __forceinline__ void swiglu16(const uint32_t (&r)[32], float st, cons
   }
 }
 
-// Shared-memory plan (offsets from a 1024-byte aligned base).
-template <int BN, bool W4, bool SWAP>
+// Shared-memory plan (offsets from a 1024-byte aligned base).  W4 here means
+// "a converter stage" (int4 or the weight-only path); KAO overrides the K atoms
+// per stage.
+template <int BN, bool W4, bool SWAP, int KAO = 0>
 struct GemmSmem {
-  static constexpr int KA = gemm_katoms(W4, false, SWAP);
+  static constexpr int KA = KAO ? KAO : gemm_katoms(W4, false, SWAP);
   static constexpr int A_ATOM = GEMM_BM * GEMM_BK;  // one 128-byte K atom of the A tile
   static constexpr int B_ATOM = BN * GEMM_BK;
   static constexpr int A_BYTES = KA * A_ATOM;
   static constexpr int B_BYTES = KA * B_ATOM;
   static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
-  static constexpr int P_BYTES = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 weight tile
-  static_assert(!W4 || KA == 1, "int4 stages hold one K atom");
+  static constexpr int P_ATOM = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 / int8 weight atom
+  static constexpr int P_BYTES = KA * P_ATOM;
   static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
   // per epilogue warp two 4 KB staging buffers (32 rows x 128 B) for output
   // stores and split-tile reductions
@@ -231,7 +237,8 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
   constexpr bool CONV = W4 || WBF;  // a converter stage between TMA and the MMA
   static_assert(!(W4 && WBF), "int4 weights have no weight-only path");
   static_assert(!(WBF && EPI == EPI_SWIGLU), "the weight-only path has no SwiGLU epilogue");
-  using SM = GemmSmem<BN, CONV, SWAP>;
+  using SM = GemmSmem<BN, CONV, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0>;
+  static_assert(!W4 || SM::KA == 1, "int4 stages hold one K atom");
   constexpr int CW = SM::CW;
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
   constexpr uint32_t IDESC = WBF ? idesc_bf16_f32(GEMM_BM, BN) : idesc_s8s8s32(GEMM_BM, BN);
@@ -334,12 +341,13 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
             // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
             const int atom = kb * KA + j;
             if (CONV && SWAP)
-              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmA, &full[s], xa(atom), ta * GEMM_BM,
-                          pol_a);
+              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES + j * SM::P_ATOM, &tmA, &full[s], xa(atom),
+                          ta * GEMM_BM, pol_a);
             else
               tma_load_2d(st + j * SM::A_ATOM, &tmA, &full[s], xa(atom), ta * GEMM_BM, pol_a);
             if (CONV && !SWAP)
-              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES, &tmB, &full[s], xb(atom), tb * BN, pol_b);
+              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES + j * SM::P_ATOM, &tmB, &full[s], xb(atom),
+                          tb * BN, pol_b);
             else
               tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, &full[s], xb(atom), tb * BN, pol_b);
           }
@@ -752,9 +760,13 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           break;
         }
         uint8_t* st = smem + s * SM::STAGE;
-        const uint8_t* packed = st + SM::A_BYTES + SM::B_BYTES;
-        uint8_t* unp = SWAP ? st : st + SM::A_BYTES;
-        for (int idx = ct; idx < WR * 4; idx += 128) {
+#pragma unroll
+        for (int j = 0; j < SM::KA; ++j) {
+        const uint8_t* packed = st + SM::A_BYTES + SM::B_BYTES + j * SM::P_ATOM;
+        uint8_t* unp = SWAP ? st + j * SM::A_ATOM : st + SM::A_BYTES + j * SM::B_ATOM;
+#pragma unroll
+        for (int i = 0; i < WR * 4 / 128; ++i) {
+          const int idx = ct + 128 * i;
           const int r = idx >> 2, pc = idx & 3;
           const uint4 pk = *reinterpret_cast<const uint4*>(packed + r * 64 + pc * 16);
           const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
@@ -787,6 +799,7 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           const int sw = r & 7;
           *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
         }
         fence_proxy_async_smem();
         mbar_arrive(&conv[s]);
