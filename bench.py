@@ -478,57 +478,77 @@ def run_ours(args, rank, world, dev):
 
 
 def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
-    """Same metric through the public API with pinned host buffers: each step
-    copies its activations host->device and its outputs device->host."""
+    """Same metric through the public API with pinned host buffers: every step
+    copies its activations host->device and its outputs device->host.
+
+    Steps are double-buffered over three streams, as a serving loop would run
+    them: step i's upload (copy-in stream) overlaps step i-1's kernels
+    (compute stream) and step i-2's download (copy-out stream).  Events order
+    each step's copy-in -> compute -> copy-out and keep a buffer from being
+    reused before the step that last used it is done.  The timed region runs
+    from the first upload to the last download."""
     ws = cr.Workspace(dev.index)
     linear = cr.convrot_int8_linear if w.weight_bits == 8 else cr.convrot_w4a8_linear
-    stream = torch.cuda.current_stream(dev)
+    swiglu = cr.convrot_int8_linear_swiglu if w.weight_bits == 8 else cr.convrot_w4a8_linear_swiglu
     steps = max(5, min(args.steps, 50))
-    if w.mlp:
-        # the block's input comes from the host and its output goes back; H
-        # stays on the device between the two GEMMs
-        host_x = [inputs[0].cpu().pin_memory()]
-        host_y = [torch.empty(w.M, layers[1].out_cols, dtype=torch.bfloat16).pin_memory()]
-        gu, down = layers
-        swiglu = cr.convrot_int8_linear_swiglu if w.weight_bits == 8 else cr.convrot_w4a8_linear_swiglu
+    # the step's inputs (one activation per input group; the MLP block's only
+    # input is x) and outputs (one per linear; the MLP block's is down_proj's)
+    ins = [inputs[0]] if w.mlp else list(inputs)
+    out_shapes = [(w.M, layers[1].out_cols)] if w.mlp else [(w.M, l.lin.N) for l in layers]
+    host_x = [x.cpu().pin_memory() for x in ins]
+    host_y = [[torch.empty(sh, dtype=torch.bfloat16).pin_memory() for sh in out_shapes] for _ in range(2)]
+    dev_x = [[torch.empty_like(x, device=dev) for x in ins] for _ in range(2)]
+    dev_y = [[torch.empty(sh, dtype=torch.bfloat16, device=dev) for sh in out_shapes] for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    up, done, down = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    for e in up + done + down:
+        e.record(torch.cuda.current_stream(dev))
 
-        def step():
-            x = host_x[0].to(dev, non_blocking=True)
-            Xq, s_tok = cr.convrot_rotate_quant_act(x, 256, norms[0], 1e-6)
+    def compute(xs, ys):
+        if w.mlp:
+            gu, dn = layers
+            Xq, s_tok = cr.convrot_rotate_quant_act(xs[0], 256, norms[0], 1e-6)
             H = swiglu(Xq, s_tok, gu.Wq, gu.s_row, workspace=ws)
             Hq, s_h = cr.convrot_rotate_quant_act(H, 256, None, 1e-6)
-            host_y[0].copy_(linear(Hq, s_h, down.Wq, down.s_row, workspace=ws), non_blocking=True)
-    else:
-        host_x = [x.cpu().pin_memory() for x in inputs]
-        host_y = [torch.empty(w.M, l.lin.N, dtype=torch.bfloat16).pin_memory() for l in layers]
-        step = None
-        if w.weight_only:
-            def step():
-                xs = [h.to(dev, non_blocking=True) for h in host_x]
-                xr = [cr.convrot_rotate_act_bf16(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
-                for li, l in enumerate(layers):
-                    host_y[li].copy_(cr.convrot_weight_only_linear(xr[l.group_in], l.Wq, l.s_row),
-                                     non_blocking=True)
+            linear(Hq, s_h, dn.Wq, dn.s_row, out=ys[0], workspace=ws)
+        elif w.weight_only:
+            xr = [cr.convrot_rotate_act_bf16(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
+            for li, l in enumerate(layers):
+                cr.convrot_weight_only_linear(xr[l.group_in], l.Wq, l.s_row, out=ys[li])
+        else:
+            qs = [cr.convrot_rotate_quant_act(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
+            for li, l in enumerate(layers):
+                linear(qs[l.group_in][0], qs[l.group_in][1], l.Wq, l.s_row, out=ys[li], workspace=ws)
 
-    def layer_step():
-        xs = [h.to(dev, non_blocking=True) for h in host_x]
-        qs = [cr.convrot_rotate_quant_act(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
-        for li, l in enumerate(layers):
-            Y = linear(qs[l.group_in][0], qs[l.group_in][1], l.Wq, l.s_row, workspace=ws)
-            host_y[li].copy_(Y, non_blocking=True)
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(done[b])            # step i-2's kernels have read dev_x[b]
+            for h, d in zip(host_x, dev_x[b]):
+                d.copy_(h, non_blocking=True)
+            up[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(up[b])
+            s_cmp.wait_event(down[b])           # step i-2's download has read dev_y[b]
+            compute(dev_x[b], dev_y[b])
+            done[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[b])
+            for d, h in zip(dev_y[b], host_y[b]):
+                h.copy_(d, non_blocking=True)
+            down[b].record(s_out)
 
-    if step is None:
-        step = layer_step
-    for _ in range(3):
-        step()
+    for i in range(4):
+        step(i)
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
-    t0.record(stream)
-    for _ in range(steps):
-        step()
-    t1.record(stream)
+    t0.record(s_in)
+    for i in range(steps):
+        step(i)
+    t1.record(s_out)
     torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1)
     if world > 1:
@@ -537,7 +557,8 @@ def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
         ms = float(t.item())
     return {"value": round(w.M * steps * world / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": sum(h.numel() * 2 for h in host_x),
-            "d2h_bytes_per_step": sum(h.numel() * 2 for h in host_y), "steps": steps}
+            "d2h_bytes_per_step": sum(h.numel() * 2 for h in host_y[0]), "steps": steps,
+            "pipelining": "double-buffered: copy-in, compute and copy-out streams ordered by events"}
 
 
 # ------------------------------------------------------------------ oracle arm
