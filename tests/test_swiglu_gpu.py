@@ -316,3 +316,20 @@ def test_convrot_mlp_class_matches_the_abi_steps(cr):
     y_f = h @ _f64(Wd).T
     rel = np.linalg.norm(_f64(y) - y_f) / np.linalg.norm(y_f)
     assert rel < 0.05, rel
+
+
+def test_w4a8_swiglu_stream_k_and_max_k(cr):
+    # int4 weights through the split-tile schedule, and the longest K the ABI takes
+    for (M, I, K) in [(768, 3200, 12288), (3, 16, 131072)]:
+        X = _rand_i8((M, K), M + 1)
+        codes = torch.randint(-8, 8, (2 * I, K), generator=torch.Generator().manual_seed(K))
+        packed = torch.from_numpy(ref.pack_int4(codes.numpy()))
+        st = _rand_scales(M, 13)
+        sgu = _rand_scales(2 * I, 14, lo=1e-3, span=2e-2)
+        H = cr.convrot_w4a8_linear_swiglu(X.cuda(), st.cuda(), packed.cuda(), sgu.cuda())
+        torch.cuda.synchronize()
+        assert cr.convrot_device_status() == 0
+        rows = np.unique(np.r_[0, M - 1, np.random.default_rng(K).integers(0, M, 8)])
+        hb, h64 = _h_ref_rows(X.numpy(), st.double().numpy(), ref.unpack_int4(packed.numpy()),
+                              sgu.double().numpy(), rows)
+        _assert_bf16_step(_f64(H)[rows], hb, h64, f"w4a8 swiglu {M}x{I}x{K}")

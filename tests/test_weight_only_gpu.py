@@ -114,3 +114,33 @@ def test_weight_only_layer_end_to_end(cr, M, K, N, group):
     # and the layer approximates the float product (weight rounding only)
     y_f = ref.rmsnorm(_f64(x), nw.double().numpy(), 1e-6) @ _f64(W).T
     assert np.linalg.norm(_f64(Y) - y_f) / np.linalg.norm(y_f) < 0.02
+
+
+@pytest.mark.parametrize("M,N,K", [(17, 136, 256), (65, 264, 512), (2, 16, 131072)])
+def test_weight_only_ragged_token_tiles_and_max_k(cr, M, N, K):
+    # partial token tiles of every width the swapped roles use, and the longest K
+    Xr, Wq, s = _operands(M, N, K)
+    Y = cr.convrot_weight_only_linear(Xr.cuda(), Wq.cuda(), s.cuda())
+    torch.cuda.synchronize()
+    assert cr.convrot_device_status() == 0
+    yb, y64 = ref.weight_only_linear(_f64(Xr), Wq.numpy(), s.double().numpy())
+    mag = (np.abs(_f64(Xr)) @ np.abs(Wq.numpy().astype(np.float64)).T) * s.double().numpy()[None, :]
+    assert np.all(np.abs(_f64(Y) - yb) <= _tol.bf16_ulp(y64) * 1.0001 + 8 * np.sqrt(K) * _tol.U * mag)
+
+
+def test_weight_only_edge_cases(cr):
+    # M = 0 is a no-op; mismatched K and a K that is not a multiple of 16 are rejected
+    Wq = torch.zeros(16, 256, dtype=torch.int8, device="cuda")
+    s = torch.ones(16, device="cuda")
+    Y = cr.convrot_weight_only_linear(torch.zeros(0, 256, dtype=torch.bfloat16, device="cuda"), Wq, s)
+    assert Y.shape == (0, 16)
+    with pytest.raises(ValueError):
+        cr.convrot_weight_only_linear(torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda"), Wq, s)
+    with pytest.raises(cr.ConvRotError):
+        cr.convrot_weight_only_linear(torch.zeros(4, 40, dtype=torch.bfloat16, device="cuda"),
+                                      torch.zeros(16, 40, dtype=torch.int8, device="cuda"), s)
+    # an all-zero weight row gives exact zeros
+    Xr, Wq2, s2 = _operands(9, 32, 512)
+    Wq2[5] = 0
+    Y2 = cr.convrot_weight_only_linear(Xr.cuda(), Wq2.cuda(), s2.cuda())
+    assert not Y2[:, 5].any()
