@@ -288,6 +288,27 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (SWAP && threadIdx.x == 64) {
+    // Decode shapes: the previous kernel (the rotate-quantise of a few
+    // tokens) occupies few SMs, so this CTA may wait here for a while.  The
+    // weights never come from that kernel: start this CTA's first stages of
+    // them towards L2 meanwhile.  A prefetch is only a hint (L2 is coherent),
+    // so it is safe before griddepcontrol.wait.  (Lane 0 of the first
+    // epilogue warp, idle until the first accumulators are ready.)
+    Schedule first;
+    first.init(a, blockIdx.x, gridDim.x);
+    Segment s0;
+    if (first.next(s0)) {
+      int ta, tb;
+      tile_coords(a, s0.tile, ta, tb);
+      const int kend = min(s0.kb1, s0.kb0 + S + GEMM_PREFETCH_ATOMS / SM::KA);
+      for (int kb = s0.kb0; kb < kend; ++kb)
+        for (int j = 0; j < SM::KA; ++j) {
+          const int atom = kb * SM::KA + j;
+          tma_prefetch_l2_2d(&tmA, (W4 || WBF) ? atom * (GEMM_BK / 2) : atom * GEMM_BK, ta * GEMM_BM);
+        }
+    }
+  }
   pdl_wait();  // operands, scales and the output may belong to the previous kernel
 
   Schedule sched;
