@@ -265,7 +265,7 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&conv[s], 128);
+      mbar_init(&conv[s], 4);  // the four converter warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tmem_full[b], 1);
@@ -823,7 +823,8 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
         }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&conv[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[s]);
       }
     }
   }
