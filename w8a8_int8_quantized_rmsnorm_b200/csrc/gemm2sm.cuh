@@ -100,6 +100,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
   uint64_t* ready = epi_sync + 2;  // SPLIT partner: the owner's stage ring is free
   uint64_t* cv_sync = epi_sync + 3;  // int4: rendezvous of the four converter warps
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 4);
+  // Signal slots (16 bytes each; SPLIT uses the first two for `ready`).
   // int4: four 16-byte signal slots.  The partner CTA's converter warps each
   // copy 16 bytes from their own slot into the leader's, completing bytes on
   // the leader's conversion barrier: an async-proxy hand-off instead of a
@@ -357,9 +358,15 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
       if (SPLIT) {
         const uint32_t other = pq ? crank - 2u : crank + 2u;
         if (ew == 0 && lane == 0) {
-          // this CTA's MMAs are complete, so its stage ring is free
+          // this CTA's MMAs are complete, so its stage ring is free: tell the
+          // other CTA with a 16-byte async copy into its signal slot, which
+          // completes bytes on its `ready` barrier (a cluster-scope release
+          // arrive would take ~0.8 us); this CTA's own `ready` completes when
+          // the other CTA's copy lands
           mbar_arrive_expect_tx(recv, SPLIT_RECV_BYTES);
-          mbar_arrive_cluster(mapa_shared(smem_addr(ready), other));
+          mbar_arrive_expect_tx(ready, 16u);
+          bulk_copy_to_cluster(mapa_shared(smem_addr(sig + 16), other), sig, 16u,
+                               mapa_shared(smem_addr(ready), other));
         }
         // stage the columns the other CTA finalises in this CTA's own ring (above
         // the receive area), in the receive layout, then copy the warp's 8 KB in
