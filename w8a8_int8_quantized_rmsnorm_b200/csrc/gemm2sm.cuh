@@ -318,7 +318,15 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
     // columns of a tile this warp finalises: its 128-column half, or in SPLIT
     // mode 64 columns of its own pair's half of the tile
     constexpr int FC = SPLIT ? 64 : 128;
+    // A finalised tile's accumulator buffer goes back to the MMA when the next
+    // tile begins: after the last tile nothing waits for it, and its
+    // cluster-scope arrive would only delay the CTA's exit.
+    int pending = -1;
     while (next_seg(seg)) {
+      if (pending >= 0) {
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&tmem_empty[pending]), lead));
+        pending = -1;
+      }
       const uint32_t b = local & 1u;
       const uint32_t use = local >> 1;
       int ta, tb;
@@ -589,7 +597,7 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
       if (!seg.partial) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(lead_tmem_empty);
+        pending = static_cast<int>(b);
       }
       ++local;
     }
