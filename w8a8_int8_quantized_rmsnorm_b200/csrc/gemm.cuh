@@ -501,21 +501,23 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           bulk_wait_group<0>();  // this warp's reductions are performed
           fence_proxy_async_global();
         }
+        // the rendezvous orders every warp's performed reductions before the
+        // counting thread's release below (one gpu-scope ordering point, not a
+        // fence in every thread)
         __syncwarp();
-        __threadfence();
         if (!epi_rendezvous()) break;
         if (et == 0) {
           const int c_lo = sk_owner(a, u_sk * a.num_kb);
           const int c_hi = sk_owner(a, (u_sk + 1) * a.num_kb - 1);
-          __threadfence();
-          const unsigned prev = atomicAdd(&a.ws_counts[u_sk], 1u);
+          const unsigned prev = atomic_add_acq_rel_gpu(&a.ws_counts[u_sk], 1u);
           const bool last = prev + 1u == static_cast<unsigned>(c_hi - c_lo + 1);
           if (last) a.ws_counts[u_sk] = 0u;  // leave the workspace clean for the next call
           *last_flag = last ? 1 : 0;
         }
         if (!epi_rendezvous()) break;
+        // the counting thread acquired the other units' sums; the rendezvous
+        // carries that to every thread of the CTA
         finalize = *last_flag != 0;
-        if (finalize) __threadfence();
       }
       if (finalize) {
         if (!SWAP) {

@@ -348,6 +348,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Atomic add with acquire-release semantics at GPU scope: orders everything
+// this thread wrote or observed before it (release) and makes everything the
+// previous arrivers released visible after it (acquire).
+__device__ __forceinline__ unsigned atomic_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Programmatic dependent launch.  A kernel launched with it may start while
 // the previous kernel on the stream is finishing: pdl_wait() returns once
 // every kernel it depends on has completed and its writes are visible, and
