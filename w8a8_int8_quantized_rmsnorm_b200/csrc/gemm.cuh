@@ -189,7 +189,10 @@ __device__ __forceinline__ void swiglu16(const uint32_t (&r)[32], float st, cons
 
 // Shared-memory plan (offsets from a 1024-byte aligned base).  W4 here means
 // "a converter stage" (int4 or the weight-only path); KAO overrides the K atoms
-// per stage.
+// per stage.  A converter stage's packed weight atom (64 bytes per row) lands
+// in the upper half of its weight atom's slot and is expanded in place to the
+// 128-byte swizzled rows the MMA reads, so a stage holds no separate packed
+// area.
 template <int BN, bool W4, bool SWAP, int KAO = 0>
 struct GemmSmem {
   static constexpr int KA = KAO ? KAO : gemm_katoms(W4, false, SWAP);
@@ -199,8 +202,9 @@ struct GemmSmem {
   static constexpr int B_BYTES = KA * B_ATOM;
   static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
   static constexpr int P_ATOM = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 / int8 weight atom
-  static constexpr int P_BYTES = KA * P_ATOM;
-  static constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int P_BYTES = KA * P_ATOM;                      // packed bytes per stage
+  static constexpr int PACKED_OFF = W_ROWS * (GEMM_BK / 2);        // inside a weight atom's slot
+  static constexpr int STAGE = A_BYTES + B_BYTES;
   // per epilogue warp two 4 KB staging buffers (32 rows x 128 B) for output
   // stores and split-tile reductions
   static constexpr int STAGING = 4 * 2 * 4096;
@@ -209,9 +213,10 @@ struct GemmSmem {
   static constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
   __host__ __device__ static int staging_offset(int stages) { return stages * STAGE; }
   __host__ __device__ static int bar_offset(int stages) { return stages * STAGE + STAGING; }
-  // full, empty, conv: stages each; tmem_full, tmem_empty: 2 each; + scalars
+  // full, empty, conv: stages each; tmem_full, tmem_empty: 2 each; drain,
+  // epi_sync, cv_sync; + scalars
   __host__ __device__ static int total(int stages) {
-    return bar_offset(stages) + (3 * GEMM_MAX_STAGES + 6) * 8 + 64;
+    return bar_offset(stages) + (3 * GEMM_MAX_STAGES + 7) * 8 + 64;
   }
 };
 
@@ -254,7 +259,8 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
   uint64_t* tmem_empty = tmem_full + 2;
   uint64_t* drain = tmem_empty + 2;
   uint64_t* epi_sync = drain + 1;  // rendezvous of the four epilogue warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_sync + 1);
+  uint64_t* cv_sync = epi_sync + 1;  // rendezvous of the four converter warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cv_sync + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -273,6 +279,7 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
     }
     mbar_init(drain, 1);
     mbar_init(epi_sync, 4);
+    mbar_init(cv_sync, 4);
     *abort_flag = 0;
     *last_flag = 0;
     fence_barrier_init();
@@ -361,16 +368,11 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           for (int j = 0; j < KA; ++j) {
             // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
             const int atom = kb * KA + j;
-            if (CONV && SWAP)
-              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES + j * SM::P_ATOM, &tmA, &full[s], xa(atom),
-                          ta * GEMM_BM, pol_a);
-            else
-              tma_load_2d(st + j * SM::A_ATOM, &tmA, &full[s], xa(atom), ta * GEMM_BM, pol_a);
-            if (CONV && !SWAP)
-              tma_load_2d(st + SM::A_BYTES + SM::B_BYTES + j * SM::P_ATOM, &tmB, &full[s], xb(atom),
-                          tb * BN, pol_b);
-            else
-              tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM, &tmB, &full[s], xb(atom), tb * BN, pol_b);
+            // a packed weight atom lands in the upper half of its slot
+            tma_load_2d(st + j * SM::A_ATOM + ((CONV && SWAP) ? SM::PACKED_OFF : 0), &tmA, &full[s],
+                        xa(atom), ta * GEMM_BM, pol_a);
+            tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM + ((CONV && !SWAP) ? SM::PACKED_OFF : 0),
+                        &tmB, &full[s], xb(atom), tb * BN, pol_b);
           }
           if (kb + pfd < seg.kb1) prefetch(ta, tb, kb + pfd);
           if (kb == win)
@@ -769,10 +771,13 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
     if (lane == 0) bulk_wait_group_read<0>();
   } else if (CONV) {
     // ------------------------------------------------------------ int4 unpack /
-    // int8 -> bf16 (WBF)
+    // int8 -> bf16 (WBF).  Each thread reads its share of every packed atom of
+    // the stage, the four warps meet (bounded), then each writes the expanded
+    // swizzled rows over the slot the packed bytes came in.
     const int ct = threadIdx.x - 192;  // 0..127
     constexpr int WR = SM::W_ROWS;
-    uint32_t it = 0;
+    constexpr int PER = WR * 4 / 128;  // 16-byte packed pieces per thread and atom
+    uint32_t it = 0, cv_phase = 0;
     bool ok = true;
     while (ok && sched.next(seg)) {
       for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
@@ -783,15 +788,34 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           break;
         }
         uint8_t* st = smem + s * SM::STAGE;
+        uint4 pks[SM::KA][PER];
 #pragma unroll
         for (int j = 0; j < SM::KA; ++j) {
-        const uint8_t* packed = st + SM::A_BYTES + SM::B_BYTES + j * SM::P_ATOM;
+          const uint8_t* packed =
+              (SWAP ? st + j * SM::A_ATOM : st + SM::A_BYTES + j * SM::B_ATOM) + SM::PACKED_OFF;
+#pragma unroll
+          for (int i = 0; i < PER; ++i) {
+            const int idx = ct + 128 * i;
+            pks[j][i] = *reinterpret_cast<const uint4*>(packed + (idx >> 2) * 64 + (idx & 3) * 16);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(cv_sync);
+        const bool met = mbar_wait(cv_sync, cv_phase & 1u, abort_flag, SITE_CONV_FULL);
+        ++cv_phase;
+        __syncwarp();
+        if (!met) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int j = 0; j < SM::KA; ++j) {
         uint8_t* unp = SWAP ? st + j * SM::A_ATOM : st + SM::A_BYTES + j * SM::B_ATOM;
 #pragma unroll
-        for (int i = 0; i < WR * 4 / 128; ++i) {
+        for (int i = 0; i < PER; ++i) {
           const int idx = ct + 128 * i;
           const int r = idx >> 2, pc = idx & 3;
-          const uint4 pk = *reinterpret_cast<const uint4*>(packed + r * 64 + pc * 16);
+          const uint4 pk = pks[j][i];
           const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
           uint32_t o[8];
 #pragma unroll
