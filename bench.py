@@ -272,7 +272,7 @@ def run_ours(args, rank, world, dev):
         l = layers[li]
         Wq, s_row = w_sets[c][li]
         if wo:
-            cr.convrot_weight_only_linear(Xq[l.group_in], Wq, s_row, out=Ys[li])
+            cr.convrot_weight_only_linear(Xq[l.group_in], Wq, s_row, out=Ys[li], workspace=ws)
             return
         (swiglu if l.swiglu else linear)(Xq[l.group_in], st[l.group_in], Wq, s_row, out=Ys[li],
                                          workspace=ws)
@@ -515,7 +515,7 @@ def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
         elif w.weight_only:
             xr = [cr.convrot_rotate_act_bf16(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
             for li, l in enumerate(layers):
-                cr.convrot_weight_only_linear(xr[l.group_in], l.Wq, l.s_row, out=ys[li])
+                cr.convrot_weight_only_linear(xr[l.group_in], l.Wq, l.s_row, out=ys[li], workspace=ws)
         else:
             qs = [cr.convrot_rotate_quant_act(xs[g], 256, norms[g], 1e-6) for g in range(len(groups))]
             for li, l in enumerate(layers):

@@ -282,17 +282,25 @@ convrot_status convrot_fold_row_scales(float* s_row, const float* smooth, int n,
  * multiplied on the tensor cores (bf16 inputs, fp32 accumulation), so Y
  * approximates x W^T with the weight's int8 rounding only.
  * x bf16 [M, K], Xr bf16 [M, K], Wq int8 [N, K], s_row fp32 [N], Y bf16 [M, N];
- * K % 16 == 0, N % 8 == 0; all 16-byte aligned.  No workspace is needed.
+ * K % 16 == 0, N % 8 == 0; all 16-byte aligned.
+ * workspace: at least convrot_weight_only_workspace_bytes(M, N, K) bytes
+ * (0: may be NULL), with the rules of convrot_int8_linear.  Decode shapes
+ * split the K range of some output tiles over two CTAs; their fp32 partial
+ * sums meet there, added at L2.  A tile never has more than two parts, and
+ * 0 + a + b is the same in either order, so results do not depend on timing.
  * convrot_weight_only_gemm_f32 writes the raw fp32 accumulators instead
  * (acc fp32 [M, N]) for accuracy checks.
  */
 convrot_status convrot_rotate_act_bf16(const void* x, int M, int K, int group,
                                        const float* norm_w, float eps, void* Xr,
                                        convrot_stream_t stream);
+size_t convrot_weight_only_workspace_bytes(int M, int N, int K);
 convrot_status convrot_weight_only_linear(const void* Xr, const int8_t* Wq, const float* s_row,
-                                          int M, int N, int K, void* Y, convrot_stream_t stream);
+                                          int M, int N, int K, void* Y, void* workspace,
+                                          size_t workspace_bytes, convrot_stream_t stream);
 convrot_status convrot_weight_only_gemm_f32(const void* Xr, const int8_t* Wq, int M, int N, int K,
-                                            float* acc, convrot_stream_t stream);
+                                            float* acc, void* workspace, size_t workspace_bytes,
+                                            convrot_stream_t stream);
 
 /*
  * Allocation-free W8A8 linear.  The model cards have no counterpart: this is

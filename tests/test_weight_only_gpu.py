@@ -57,8 +57,10 @@ def test_rotate_act_bf16(cr, M, K, group, norm):
     assert np.all(err <= _tol.bf16_ulp(v) * 1.0001 + 2 * e32), f"worst {np.max(err - _tol.bf16_ulp(v)):.3e}"
 
 
+# (16, 20480, 1024) and (100, 20480, 4096) split the K range of some tiles over
+# two CTAs (stream-K with fp32 partial sums); the others run whole tiles
 SHAPES = [(1, 256, 256), (16, 1024, 4096), (40, 520, 1040), (128, 4096, 4096), (129, 264, 512),
-          (512, 4096, 4096), (1000, 1032, 2080)]
+          (512, 4096, 4096), (1000, 1032, 2080), (16, 20480, 1024), (100, 20480, 4096)]
 
 
 def _operands(M, N, K):
@@ -144,3 +146,22 @@ def test_weight_only_edge_cases(cr):
     Wq2[5] = 0
     Y2 = cr.convrot_weight_only_linear(Xr.cuda(), Wq2.cuda(), s2.cuda())
     assert not Y2[:, 5].any()
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 20480, 1024), (100, 20480, 4096)])
+def test_weight_only_split_tiles_deterministic(cr, M, N, K):
+    """Split tiles have at most two fp32 parts, so repeated calls agree bit for
+    bit whatever the order the parts arrive in; the workspace is zero again."""
+    Xr, Wq, s = _operands(M, N, K)
+    assert cr.convrot_weight_only_workspace_bytes(M, N, K) > 0
+    ws = cr.Workspace()
+    Xd, Wd, sd = Xr.cuda(), Wq.cuda(), s.cuda()
+    ys = [cr.convrot_weight_only_linear(Xd, Wd, sd, workspace=ws) for _ in range(6)]
+    acc = [cr.convrot_weight_only_gemm_f32(Xd, Wd, workspace=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert cr.convrot_device_status() == 0
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
+    for a in acc[1:]:
+        assert torch.equal(a, acc[0])
+    assert int(ws.buf.count_nonzero()) == 0

@@ -22,7 +22,8 @@ __all__ = [
     "convrot_w4a8_linear", "convrot_int8_linear_noalloc", "convrot_int8_gemm_s32", "convrot_w4a8_gemm_s32",
     "convrot_swiglu_workspace_bytes", "convrot_int8_linear_swiglu", "convrot_w4a8_linear_swiglu",
     "convrot_interleave_gate_up", "convrot_fold_row_scales",
-    "convrot_rotate_act_bf16", "convrot_weight_only_linear", "convrot_weight_only_gemm_f32",
+    "convrot_rotate_act_bf16", "convrot_weight_only_workspace_bytes", "convrot_weight_only_linear",
+    "convrot_weight_only_gemm_f32",
     "Workspace", "ConvRotLinear", "ConvRotFusedLinear", "ConvRotMLP",
 ]
 
@@ -266,21 +267,27 @@ def _wo_check(Xr, Wq):
     return Xr.shape[0], Wq.shape[0], Xr.shape[1]
 
 
-def convrot_weight_only_linear(Xr, Wq, s_row, out=None):
+def convrot_weight_only_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().convrot_weight_only_workspace_bytes(M, N, K))
+
+
+def convrot_weight_only_linear(Xr, Wq, s_row, out=None, workspace: Optional[Workspace] = None):
     """Y = bf16(s_row * (Xr @ Wq^T)) on rotated bf16 activations, int8 weights."""
     M, N, K = _wo_check(Xr, Wq)
     _need(s_row, torch.float32, "s_row", 1)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xr.device) if out is None else out
+    ws, wn = _workspace(Xr.device, convrot_weight_only_workspace_bytes(M, N, K), workspace)
     _check("convrot_weight_only_linear", lib().convrot_weight_only_linear(
-        _ptr(Xr), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), _stream(Xr.device)))
+        _ptr(Xr), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), ws, wn, _stream(Xr.device)))
     return Y
 
 
-def convrot_weight_only_gemm_f32(Xr, Wq):
+def convrot_weight_only_gemm_f32(Xr, Wq, workspace: Optional[Workspace] = None):
     M, N, K = _wo_check(Xr, Wq)
     acc = torch.empty(M, N, dtype=torch.float32, device=Xr.device)
+    ws, wn = _workspace(Xr.device, convrot_weight_only_workspace_bytes(M, N, K), workspace)
     _check("convrot_weight_only_gemm_f32", lib().convrot_weight_only_gemm_f32(
-        _ptr(Xr), _ptr(Wq), M, N, K, _ptr(acc), _stream(Xr.device)))
+        _ptr(Xr), _ptr(Wq), M, N, K, _ptr(acc), ws, wn, _stream(Xr.device)))
     return acc
 
 
@@ -394,7 +401,7 @@ class ConvRotLinear:
         if self.weight_bits != 8:
             raise ValueError("the weight-only path takes int8 weights")
         Xr = convrot_rotate_act_bf16(x, self.group, self.norm_w, self.eps)
-        return convrot_weight_only_linear(Xr, self.Wq, self.s_row, out)
+        return convrot_weight_only_linear(Xr, self.Wq, self.s_row, out, self.workspace)
 
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         Xq, s_tok = convrot_rotate_quant_act(x, self.group, self.norm_w, self.eps)

@@ -58,9 +58,11 @@ SIGNATURES = {
     "convrot_fold_row_scales": (c_int, [c_void_p, c_void_p, c_int, c_void_p]),
     "convrot_rotate_act_bf16": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_float, c_void_p,
                                         c_void_p]),
+    "convrot_weight_only_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
     "convrot_weight_only_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
-                                           c_void_p]),
-    "convrot_weight_only_gemm_f32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
+                                           c_void_p, c_size_t, c_void_p]),
+    "convrot_weight_only_gemm_f32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,
+                                             c_void_p, c_size_t, c_void_p]),
     "convrot_int8_linear_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                             c_int, c_void_p, c_void_p]),
     "convrot_int8_gemm_s32": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p,

@@ -303,8 +303,10 @@ int pick_bn_swap(int M) {
 // `clusters4` is the number of co-resident four-CTA clusters of the split
 // pair kernel (0 if unavailable).
 // wbf: the weight-only path (bf16 activations, int8 weights expanded to bf16,
-// fp32 accumulators): single-CTA tiles, 64 K elements per stage, plain waves
-// only (its fp32 partial sums have no split-tile reduction).
+// fp32 accumulators): single-CTA tiles, 64 K elements per stage; stream-K
+// only for the swapped roles and only where every split tile has at most two
+// parts (each unit's share is at least a whole tile), so that the fp32 sum of
+// the parts does not depend on their order.
 GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int clusters4,
                    bool wbf = false) {
   GemmPlan p{};
@@ -348,7 +350,8 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   const long long sk_total = static_cast<long long>(sk_tiles) * p.num_kb;
   const long long t_sk = static_cast<long long>(p.dp_tiles / p.grid) * p.num_kb +
                          (sk_total + p.grid - 1) / p.grid + fixup_stages(p.swap, p.bn);
-  if (wbf || t_dp <= t_sk) {
+  const bool two_parts = sk_tiles * p.num_kb / p.grid >= p.num_kb;
+  if ((wbf && (!p.swap || !two_parts)) || t_dp <= t_sk) {
     p.dp_tiles = p.num_tiles;
     sk_tiles = 0;
   }
@@ -516,10 +519,14 @@ convrot_status launch_wbf(bool swap, int bn, const CUtensorMap& ma, const CUtens
 // Weight-only path: Xr bf16 [M, K] (rotated activations), Wq int8 [N, K];
 // out bf16 Y = (Xr Wq^T) * s_row, or raw fp32 accumulators (f32_out).
 convrot_status run_gemm_wbf(const void* Xr, const int8_t* Wq, const float* s_row, int M, int N,
-                            int K, void* out, bool f32_out, cudaStream_t st) {
+                            int K, void* out, bool f32_out, void* workspace, size_t workspace_bytes,
+                            cudaStream_t st) {
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
   const GemmPlan p = plan_gemm(M, N, K, d.sms, 0, false, 0, true);
+  const size_t need = ws_bytes(p);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return CONVROT_ERR_WORKSPACE;
+  if (need > 0 && !aligned(workspace, 256)) return CONVROT_ERR_ALIGN;
   const int bn = p.bn;
   CUtensorMap mx, mw, my;
   std::memset(&my, 0, sizeof(my));
@@ -551,6 +558,12 @@ convrot_status run_gemm_wbf(const void* Xr, const int8_t* Wq, const float* s_row
   a.num_tiles = p.num_tiles;
   a.num_kb = p.num_kb;
   a.dp_tiles = p.dp_tiles;
+  a.sk_iters = p.sk_iters;
+  a.sk_q = p.sk_q;
+  a.sk_r = p.sk_r;
+  a.ws_counts = need ? static_cast<unsigned*>(workspace) : nullptr;
+  a.ws_acc = need ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + kCounterBytes)
+                  : nullptr;
   a.s_tok = nullptr;
   a.s_row = s_row;
   a.srow_vec = (s_row != nullptr && aligned(s_row, 16)) ? 1 : 0;
@@ -926,8 +939,16 @@ convrot_status convrot_rotate_act_bf16(const void* x, int M, int K, int group,
                 : launch_rowquant_pre<PRE_NONE, QK_BF16>(a, group, as_cuda(stream));
 }
 
+size_t convrot_weight_only_workspace_bytes(int M, int N, int K) {
+  if (check_gemm_shape(M, N, K, false) != CONVROT_OK || M == 0 || N == 0) return 0;
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return 0;
+  return ws_bytes(plan_gemm(M, N, K, d.sms, 0, false, 0, true));
+}
+
 static convrot_status weight_only_common(const void* Xr, const int8_t* Wq, const float* s_row,
                                          int M, int N, int K, void* out, bool f32_out,
+                                         void* workspace, size_t workspace_bytes,
                                          convrot_stream_t stream) {
   const convrot_status sh = check_gemm_shape(M, N, K, false);
   if (sh != CONVROT_OK) return sh;
@@ -935,17 +956,21 @@ static convrot_status weight_only_common(const void* Xr, const int8_t* Wq, const
   if (!Xr || !Wq || !out || (!f32_out && !s_row)) return CONVROT_ERR_NULL;
   if (!aligned(Xr, 16) || !aligned(Wq, 16) || !aligned(out, 16) || (s_row && !aligned(s_row, 4)))
     return CONVROT_ERR_ALIGN;
-  return run_gemm_wbf(Xr, Wq, s_row, M, N, K, out, f32_out, as_cuda(stream));
+  return run_gemm_wbf(Xr, Wq, s_row, M, N, K, out, f32_out, workspace, workspace_bytes,
+                      as_cuda(stream));
 }
 
 convrot_status convrot_weight_only_linear(const void* Xr, const int8_t* Wq, const float* s_row,
-                                          int M, int N, int K, void* Y, convrot_stream_t stream) {
-  return weight_only_common(Xr, Wq, s_row, M, N, K, Y, false, stream);
+                                          int M, int N, int K, void* Y, void* workspace,
+                                          size_t workspace_bytes, convrot_stream_t stream) {
+  return weight_only_common(Xr, Wq, s_row, M, N, K, Y, false, workspace, workspace_bytes, stream);
 }
 
 convrot_status convrot_weight_only_gemm_f32(const void* Xr, const int8_t* Wq, int M, int N, int K,
-                                            float* acc, convrot_stream_t stream) {
-  return weight_only_common(Xr, Wq, nullptr, M, N, K, acc, true, stream);
+                                            float* acc, void* workspace, size_t workspace_bytes,
+                                            convrot_stream_t stream) {
+  return weight_only_common(Xr, Wq, nullptr, M, N, K, acc, true, workspace, workspace_bytes,
+                            stream);
 }
 
 convrot_status convrot_interleave_gate_up(const void* Wg, const void* Wu, int I,

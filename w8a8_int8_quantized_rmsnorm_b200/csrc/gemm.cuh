@@ -489,7 +489,10 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            bulk_reduce_add_s32(acc_tile + (c * 4 + q) * 32 * CW, stage_buf, 128 * CW);
+            if (WBF)
+              bulk_reduce_add_f32(acc_tile + (c * 4 + q) * 32 * CW, stage_buf, 128 * CW);
+            else
+              bulk_reduce_add_s32(acc_tile + (c * 4 + q) * 32 * CW, stage_buf, 128 * CW);
             bulk_commit_group();
           }
         }

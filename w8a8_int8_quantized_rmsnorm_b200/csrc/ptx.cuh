@@ -151,6 +151,15 @@ __device__ __forceinline__ void bulk_reduce_add_s32(void* dst_global, const void
                : "memory");
 }
 
+// The same for fp32 (the adds happen at L2 in arrival order).
+__device__ __forceinline__ void bulk_reduce_add_f32(void* dst_global, const void* src_smem,
+                                                    uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   dst_global),
+               "r"(smem_addr(src_smem)), "r"(bytes)
+               : "memory");
+}
+
 // Orders this thread's completed async-proxy global writes before its later
 // generic-proxy memory operations.
 __device__ __forceinline__ void fence_proxy_async_global() {
