@@ -799,7 +799,10 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
 #pragma unroll
           for (int i = 0; i < PER; ++i) {
             const int idx = ct + 128 * i;
-            pks[j][i] = *reinterpret_cast<const uint4*>(packed + (idx >> 2) * 64 + (idx & 3) * 16);
+            // explicit shared-memory loads and stores schedule better for the
+            // 256-row tiles, generic ones for the decode tiles (measured)
+            const uint8_t* src = packed + (idx >> 2) * 64 + (idx & 3) * 16;
+            pks[j][i] = SWAP ? *reinterpret_cast<const uint4*>(src) : ld_shared_v4(src);
           }
         }
         __syncwarp();
@@ -847,8 +850,15 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
             }
           }
           const int sw = r & 7;
-          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(unp + r * 128 + (((2 * pc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          uint8_t* d0 = unp + r * 128 + (((2 * pc) ^ sw) << 4);
+          uint8_t* d1 = unp + r * 128 + (((2 * pc + 1) ^ sw) << 4);
+          if (SWAP) {
+            *reinterpret_cast<uint4*>(d0) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(d1) = make_uint4(o[4], o[5], o[6], o[7]);
+          } else {
+            st_shared_v4(d0, o[0], o[1], o[2], o[3]);
+            st_shared_v4(d1, o[4], o[5], o[6], o[7]);
+          }
         }
         }
         fence_proxy_async_smem();
