@@ -37,6 +37,26 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(values, world: int, device):
+    """Each entry's largest value over all ranks: a multi-rank measurement
+    takes the slowest rank's device time.  One rank: the values themselves.
+    Works on any process group (nccl on GPUs, gloo on CPU)."""
+    vals = [float(v) for v in values]
+    if world <= 1:
+        return vals
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(units_per_rank_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the (max over
+    ranks) elapsed time.  Every rank runs an independent replica of the same
+    per-rank work (weak scaling)."""
+    return units_per_rank_step * steps * world / (ms / 1e3)
 METRIC = "ConvRot W8A8 linear TOPS and tokens/s vs INT8 tensor & HBM roofline"
 DEFAULT_WORKLOAD = "down_proj_m512"
 # dense int8 tensor peak = measured dense bf16 peak x the nominal int8:bf16 ratio (4.5 / 2.25)
@@ -361,11 +381,7 @@ def run_ours(args, rank, world, dev):
     clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
     status = cr.convrot_device_status(dev.index)
     if status:
         raise RuntimeError(f"device error word {status:#x} in the timed region")
@@ -375,10 +391,7 @@ def run_ours(args, rank, world, dev):
     k1_region_ms = timed(k1_only, args.steps, k1_graph)
     run(k2_only, args.steps, k2_graph)
     k2_region_ms = timed(k2_only, args.steps, k2_graph)
-    if world > 1:
-        t = torch.tensor([k1_region_ms, k2_region_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        k1_region_ms, k2_region_ms = (float(v) for v in t.tolist())
+    k1_region_ms, k2_region_ms = max_over_ranks([k1_region_ms, k2_region_ms], world, dev)
     status = cr.convrot_device_status(dev.index)
     if status:
         raise RuntimeError(f"device error word {status:#x} in a kernel timing region")
@@ -388,7 +401,6 @@ def run_ours(args, rank, world, dev):
     k1_avg = statistics.mean(k1_ms) / n_k1  # per launch
     k2_avg = statistics.mean(k2_ms) / n_k2
 
-    tokens = w.M * args.steps * world
     ops = w.ops() * args.steps * world
     secs = elapsed_ms / 1e3
     # algorithmic bytes: K1 reads bf16 and writes int8 codes + scales (bf16 on
@@ -426,7 +438,7 @@ def run_ours(args, rank, world, dev):
 
     result = {
         "metric": METRIC,
-        "value": round(tokens / secs, 1),
+        "value": round(job_throughput(w.M, args.steps, world, elapsed_ms), 1),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -550,12 +562,8 @@ def e2e_ours(cr, args, w, groups, inputs, norms, layers, dev, world):
         step(i)
     t1.record(s_out)
     torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(w.M * steps * world / (ms / 1e3), 1), "unit": "tokens/s",
+    ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
+    return {"value": round(job_throughput(w.M, steps, world, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": sum(h.numel() * 2 for h in host_x),
             "d2h_bytes_per_step": sum(h.numel() * 2 for h in host_y[0]), "steps": steps,
             "pipelining": "double-buffered: copy-in, compute and copy-out streams ordered by events"}
