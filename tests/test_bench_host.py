@@ -1,0 +1,82 @@
+"""Host-side rules of bench.py and of the committed profile summaries.
+
+* A DRAM-traffic figure from an ncu capture is reported only while the
+  kernel sources still hash to the capture's source hash; after any kernel
+  change the bench reports traffic as null.
+* Every profile summary gives the command that produced it: ncu with
+  --clock-control none, running bench.py (a committed file) with options the
+  bench accepts, and each workload it names exists.
+"""
+import glob
+import json
+import os
+import re
+import shlex
+
+import pytest
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_traffic_only_for_matching_sources(monkeypatch):
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        t = json.load(f)
+    entry = t["down_proj_m512"]["gemm"]
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: entry["source_sha"])
+    assert bench.profiled_traffic("gemm", "down_proj_m512") == entry["dram_bytes_per_launch"]
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
+    assert bench.profiled_traffic("gemm", "down_proj_m512") is None
+    # an unprofiled kernel or workload has no figure
+    assert bench.profiled_traffic("gemm", "no_such_workload") is None
+
+
+def test_source_hash_covers_every_kernel_file(tmp_path, monkeypatch):
+    """The hash changes when any file of the kernel sources changes."""
+    src = os.path.join(ROOT, "w8a8_int8_quantized_rmsnorm_b200", "csrc")
+    fake = tmp_path / "w8a8_int8_quantized_rmsnorm_b200" / "csrc"
+    fake.mkdir(parents=True)
+    for name in sorted(os.listdir(src)):
+        with open(os.path.join(src, name), "rb") as f:
+            (fake / name).write_bytes(f.read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_sha()
+    first = sorted(os.listdir(fake))[0]
+    (fake / first).write_bytes((fake / first).read_bytes() + b"\n")
+    assert bench.kernel_source_sha() != h0
+
+
+def _commands(text):
+    """The shell commands of a summary: indented lines, backslash-joined."""
+    lines, cur = [], ""
+    for ln in text.splitlines():
+        if not ln.startswith("    "):
+            if cur:
+                lines.append(cur)
+                cur = ""
+            continue
+        part = ln.strip()
+        cur = (cur + " " + part[:-1].strip()) if part.endswith("\\") else (cur + " " + part)
+        if not part.endswith("\\"):
+            lines.append(cur.strip())
+            cur = ""
+    return [c for c in lines if c]
+
+
+@pytest.mark.parametrize("path", sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))),
+                         ids=os.path.basename)
+def test_profile_commands_run_committed_files(path, monkeypatch):
+    with open(path) as f:
+        cmds = _commands(f.read())
+    ncu = [c for c in cmds if "ncu " in c]
+    assert ncu, "a profile summary names the ncu command that produced it"
+    for c in ncu:
+        assert "--clock-control none" in c
+        prog = re.split(r"\s[>&|]", c[c.index("python "):])[0]
+        argv = shlex.split(prog)
+        assert argv[1] == "bench.py" and os.path.exists(os.path.join(ROOT, argv[1]))
+        # the bench accepts the options (argparse exits on an unknown one)
+        monkeypatch.setattr("sys.argv", argv[1:])
+        args = bench.parse()
+        assert args.workload in bench.workloads.WORKLOADS
