@@ -88,6 +88,14 @@ def test_validation_before_any_launch(lib):
     assert lib.convrot_selftest_wait_timeout(100000001, None) == 2
     # calibration may not fold in place
     assert lib.convrot_smoothquant_calibrate(A, 4, 512, A, 1e-6, A, 8, 0.5, A, A, None) == 4
+    # weight-only path: shapes, pointers and alignment before any device query
+    assert lib.convrot_weight_only_linear(A, A, A, 4, 12, 512, A, None, 0, None) == 2   # N % 8
+    assert lib.convrot_weight_only_linear(A, A, A, 4, 16, 40, A, None, 0, None) == 2    # K % 16
+    assert lib.convrot_weight_only_linear(A, A, None, 4, 16, 512, A, None, 0, None) == 1  # s_row
+    assert lib.convrot_weight_only_gemm_f32(A, A, 4, 16, 512, None, None, 0, None) == 1
+    assert lib.convrot_weight_only_linear(_p(0x10008), A, A, 4, 16, 512, A, None, 0, None) == 3
+    assert lib.convrot_weight_only_linear(None, None, None, 0, 16, 512, None, None, 0, None) == 0
+    assert lib.convrot_weight_only_workspace_bytes(4, 12, 512) == 0  # invalid shape: no size
 
 
 def test_binding_refuses_cpu_tensors():
