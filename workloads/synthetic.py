@@ -26,8 +26,7 @@ CUDA generator instead (same seeds, different stream of numbers).
 from __future__ import annotations
 
 import dataclasses
-import math
-from typing import List, Optional, Tuple
+from typing import Optional, Tuple
 
 import torch
 
