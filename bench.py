@@ -76,6 +76,8 @@ def parse():
                     help="time eager ABI calls instead of replaying captured launches")
     ap.add_argument("--copies", type=int, default=0,
                     help="input copies rotated through to defeat L2 (0 = enough for 3x L2)")
+    ap.add_argument("--no-library-reference", action="store_true",
+                    help="skip timing torch._int_mm at 8192^3 (same-box context figure)")
     return ap.parse_args()
 
 
@@ -651,6 +653,30 @@ def blas_threads():
         return os.cpu_count()
 
 
+def library_int8_reference(dev, peak_tops, n=8192, reps=20):
+    """A library int8 GEMM on the same GPU for context: torch._int_mm on
+    n x n x n int8 operands (int32 result), timed with CUDA events after
+    warm-up.  Not the target, and not part of the hot path."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        torch._int_mm(a, b)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    tops = 2.0 * n ** 3 / (ms / 1e3) / 1e12
+    del a, b
+    return {"op": "torch._int_mm", "shape": [n, n, n], "ms": round(ms, 4),
+            "tops": round(tops, 1), "frac_of_int8_peak": round(tops / peak_tops, 4)}
+
+
 def cpu_baseline(w, target_s=10.0):
     """The oracle as it stands on the host cores, on a bounded sample."""
     sample = min(w.M, 64 if w.layers == 1 else 16)
@@ -720,6 +746,10 @@ def main():
     try:
         res = run_ours(args, rank, world, dev)
         if rank == 0:
+            if not args.no_library_reference:
+                peaks = load_peaks()
+                res["library_reference"] = library_int8_reference(
+                    dev, INT8_PER_BF16 * peaks["bf16_tflops"])
             if not args.no_cpu_baseline:
                 res["cpu_baseline"] = cpu_baseline(workloads.WORKLOADS[args.workload])
             print(json.dumps(res), flush=True)
