@@ -677,10 +677,7 @@ def library_int8_reference(dev, peak_tops, n=8192, reps=20):
             "tops": round(tops, 1), "frac_of_int8_peak": round(tops / peak_tops, 4)}
 
 
-def cpu_baseline(w, target_s=10.0):
-    """The oracle as it stands on the host cores, on a bounded sample."""
-    sample = min(w.M, 64 if w.layers == 1 else 16)
-    run = oracle_step_runner(w, sample)
+def _time_oracle(run, target_s):
     run()  # warm
     reps, t = 0, 0.0
     t0 = time.perf_counter()
@@ -689,13 +686,30 @@ def cpu_baseline(w, target_s=10.0):
         reps += 1
         t = time.perf_counter() - t0
         if t >= target_s or reps >= 1000:
-            break
+            return reps, t
+
+
+def cpu_baseline(w, target_s=10.0, single_s=3.0):
+    """The oracle as it stands on the host cores, on a bounded sample; then
+    the same sample on one BLAS thread."""
+    sample = min(w.M, 64 if w.layers == 1 else 16)
+    run = oracle_step_runner(w, sample)
+    reps, t = _time_oracle(run, target_s)
     per_tok = t / (reps * sample * w.layers)
-    return {"value": round(1.0 / per_tok, 2), "unit": "tokens/s", "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": f"{sample} tokens of {w.name} x {reps} repetitions "
-                      f"({t:.1f} s; float64 numpy, every linear of the step"
-                      + (f", 1 of {w.layers} layers, scaled" if w.layers > 1 else "") + ")"}
+    res = {"value": round(1.0 / per_tok, 2), "unit": "tokens/s", "cores": blas_threads(),
+           "kind": "oracle",
+           "sample": f"{sample} tokens of {w.name} x {reps} repetitions "
+                     f"({t:.1f} s; float64 numpy, every linear of the step"
+                     + (f", 1 of {w.layers} layers, scaled" if w.layers > 1 else "") + ")"}
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return res
+    with threadpool_limits(limits=1, user_api="blas"):
+        reps1, t1 = _time_oracle(run, single_s)
+    res["single_thread"] = {"value": round(reps1 * sample * w.layers / t1, 2), "unit": "tokens/s",
+                            "cores": 1, "sample": f"the same sample x {reps1} repetitions ({t1:.1f} s)"}
+    return res
 
 
 def run_reference(args, rank, world):

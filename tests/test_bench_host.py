@@ -80,3 +80,13 @@ def test_profile_commands_run_committed_files(path, monkeypatch):
         monkeypatch.setattr("sys.argv", argv[1:])
         args = bench.parse()
         assert args.workload in bench.workloads.WORKLOADS
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    """The oracle's CPU baseline, on a tiny budget: the multi-threaded figure
+    and the single-thread one, both in tokens/s of the workload."""
+    w = bench.workloads.WORKLOADS["single_linear_m32"]
+    r = bench.cpu_baseline(w, target_s=0.2, single_s=0.2)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
+    assert r["cores"] >= 1
+    assert r["single_thread"]["cores"] == 1 and r["single_thread"]["value"] > 0
