@@ -5,15 +5,18 @@ One step = one pass of the per-token hot path over one batch of synthetic
 input: the rotate-quantise kernel (with the fused RMSNorm when the workload has
 one) and the tcgen05 W8A8 GEMM with its dequant epilogue.  Weight preparation
 (SmoothQuant calibration, rotation, per-row quantisation) is offline and not
-timed.  The default workload is the down-proj shaped linear: 512 tokens,
-K = 12288, N = 4096, RMSNorm with folded SmoothQuant scales.
+timed.  The default workload is the largest single-GPU W8A8 configuration:
+the fused gate+up projection at 8192 tokens (K = 4096, N = 24576).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle, timed on the host
 
-Under torchrun every rank runs an independent replica (the linear has no data
-exchange); the timed region is bracketed by barriers and the max over ranks
-is reported.  Rank 0 prints one JSON line.
+The K timed steps are captured as one CUDA graph.  That graph is replayed
+until at least MIN_TIMED_MS have passed (every replay is exactly K steps,
+bracketed by a barrier and a device synchronisation); the median replay gives
+ms_per_step.  Under torchrun every rank runs an independent replica (the
+linear has no data exchange) and the max over ranks of the median is
+reported.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -58,7 +61,12 @@ def job_throughput(units_per_rank_step: int, steps: int, world: int, ms: float) 
     per-rank work (weak scaling)."""
     return units_per_rank_step * steps * world / (ms / 1e3)
 METRIC = "ConvRot W8A8 linear TOPS and tokens/s vs INT8 tensor & HBM roofline"
-DEFAULT_WORKLOAD = "down_proj_m512"
+DEFAULT_WORKLOAD = "gate_up_m8192"
+# the timed graph (K steps) is replayed until at least this much device time
+# has passed; the median replay is reported
+MIN_TIMED_MS = 400.0
+MIN_REPLAYS = 5
+MAX_REPLAYS = 400
 # dense int8 tensor peak = measured dense bf16 peak x the nominal int8:bf16 ratio (4.5 / 2.25)
 INT8_PER_BF16 = 2.0
 
@@ -93,10 +101,18 @@ def load_peaks():
             "source": "fallback"}
 
 
-def kernel_source_sha():
+# the sources each reported kernel is built from: its kernel header, the PTX
+# helpers and the ABI file that plans and launches it
+KERNEL_SOURCES = {
+    "gemm": ("gemm.cuh", "gemm2sm.cuh", "ptx.cuh", "convrot_abi.cu"),
+    "rotate_quant_act": ("rowquant.cuh", "ptx.cuh", "convrot_abi.cu"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "w8a8_int8_quantized_rmsnorm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -105,16 +121,25 @@ def kernel_source_sha():
 
 def profiled_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel sources changed since the counters were taken."""
+    kernel's sources changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         t = json.load(f)
     e = t.get(workload, {}).get(kernel)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def agreed_replays(first_ms: float, world: int, device) -> int:
+    """How many times the K-step region is replayed: enough for MIN_TIMED_MS
+    of device time at the slowest rank's first replay, within [MIN_REPLAYS,
+    MAX_REPLAYS].  Every rank gets the same count, so every rank takes the
+    same collective steps."""
+    first = max_over_ranks([first_ms], world, device)[0]
+    return int(min(MAX_REPLAYS, max(MIN_REPLAYS, math.ceil(MIN_TIMED_MS / max(first, 1e-3)))))
 
 
 class ClockSampler:
@@ -358,6 +383,21 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize(dev)
         return a.elapsed_time(b)
 
+    def replays(fn, n, graph, sync_ranks):
+        """Replays the K-step region until MIN_TIMED_MS of device time have
+        passed (at least MIN_REPLAYS times); every replay is timed on its own
+        between two events on the launching stream.  The replay count is agreed
+        over ranks from the first replay, so every rank takes the same
+        collective steps.  Returns (median ms, every replay's ms)."""
+        def one():
+            if sync_ranks and world > 1:
+                torch.distributed.barrier()
+            return timed(fn, n, graph)
+        times = [one()]
+        for _ in range(agreed_replays(times[0], world, dev) - 1):
+            times.append(one())
+        return statistics.median(times), times
+
     warm_graph = region(step, args.warmup)
     timed_graph = region(step, args.steps)
     k1_graph = region(k1_only, args.steps)
@@ -369,30 +409,24 @@ def run_ours(args, rank, world, dev):
     if status:
         raise RuntimeError(f"device error word {status:#x} after warm-up")
 
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
     time.sleep(0.3)
-    t0.record(stream)
-    run(step, args.steps, timed_graph)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
+    median_ms, step_times = replays(step, args.steps, timed_graph, True)
     clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
+    elapsed_ms = max_over_ranks([median_ms], world, dev)[0]
     status = cr.convrot_device_status(dev.index)
     if status:
         raise RuntimeError(f"device error word {status:#x} in the timed region")
 
-    # per-kernel regions (each replayed once untimed first: graph upload)
-    run(k1_only, args.steps, k1_graph)
-    k1_region_ms = timed(k1_only, args.steps, k1_graph)
-    run(k2_only, args.steps, k2_graph)
-    k2_region_ms = timed(k2_only, args.steps, k2_graph)
+    # per-kernel regions, timed the same way (median of replays)
+    k1_region_ms, _ = replays(k1_only, args.steps, k1_graph, False)
+    k2_region_ms, _ = replays(k2_only, args.steps, k2_graph, False)
     k1_region_ms, k2_region_ms = max_over_ranks([k1_region_ms, k2_region_ms], world, dev)
     status = cr.convrot_device_status(dev.index)
     if status:
@@ -446,6 +480,7 @@ def run_ours(args, rank, world, dev):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(elapsed_ms / args.steps, 5),
+        "timed_replays": len(step_times),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -461,9 +496,12 @@ def run_ours(args, rank, world, dev):
                if w.mlp else {}),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "launch": ("eager ABI calls" if timed_graph is None else
-                       "the K timed steps' ABI calls captured as one CUDA graph, replayed once"),
+                       "the K timed steps' ABI calls captured as one CUDA graph"),
+            "timing": (f"{len(step_times)} replays of the K-step region, each timed between two "
+                       f"events; median reported (min {min(step_times):.4f} ms, max "
+                       f"{max(step_times):.4f} ms per replay, {sum(step_times):.1f} ms in total)"),
             "kernel_timing": ("each kernel's K * launches_per_step launches timed alone as one "
-                              "region (same inputs and copies) between two events"),
+                              "region (same inputs and copies), replayed the same way; median"),
             "l2": (f"{copies} rotating copies of the step's inputs "
                    f"({copies * step_bytes / 1e6:.0f} MB > L2)") if copies > 1
                   else f"step inputs {step_bytes / 1e6:.0f} MB > 2x L2",
@@ -483,7 +521,7 @@ def run_ours(args, rank, world, dev):
                      "algorithmic_bytes_per_step": k2_bytes, "ops_per_step": k2_ops},
         },
         "kernels_sum_ms_per_step": round((k1_region_ms + k2_region_ms) / args.steps, 5),
-        "gpu_launches": (n_k1 + n_k2) * args.steps,
+        "gpu_launches": (n_k1 + n_k2) * args.steps * len(step_times),
         "clocks": clk,
     }
     if not args.no_e2e:

@@ -202,10 +202,12 @@ size_t convrot_linear_workspace_bytes(int M, int N, int K, int weight_bits);
  * workspace: device buffer of at least convrot_linear_workspace_bytes(M, N,
  * K, 8) bytes, zero-filled before its first use.  Output tiles whose K range
  * is split across CTAs are summed there: one int32 accumulator and one
- * arrival counter per such tile.  Every call that returns CONVROT_OK leaves
+ * arrival counter per such tile.  Every call whose kernels complete leaves
  * the whole buffer zero-filled again, so it can be passed to later calls of
- * any shape without clearing.  Calls that share one workspace must not run
- * concurrently.
+ * any shape without clearing.  A call whose kernel gave up on a bounded wait
+ * (reported later by convrot_device_status as CONVROT_ERR_DEVICE_TIMEOUT)
+ * may leave partial sums behind: zero-fill the workspace again after such a
+ * report.  Calls that share one workspace must not run concurrently.
  */
 convrot_status convrot_int8_linear(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
                                    const float* s_row, int M, int N, int K, void* Y,
@@ -316,8 +318,11 @@ convrot_status convrot_weight_only_gemm_f32(const void* Xr, const int8_t* Wq, in
  *  - Shapes whose workspace exceeds 24 MiB are rejected with
  *    CONVROT_ERR_WORKSPACE (on a 148-SM B200 every M <= 128 fits; larger M
  *    with tiles split across CTAs does not - use convrot_int8_linear).
- *  - All calls on a device share the array: each call clears the part it
- *    uses (which must start at zero), and calls that overlap on the GPU race.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents.  What must start at zero (split-tile counters and partial
+ *    sums) is cleared at set-up, left zero by every call that completes, and
+ *    cleared again by the first call after convrot_device_status reported
+ *    CONVROT_ERR_DEVICE_TIMEOUT.  Calls that overlap on the GPU race on it.
  * Arguments, layouts and return codes otherwise as convrot_int8_linear.
  */
 convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const float* s_tok, const int8_t* Wq,

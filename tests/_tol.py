@@ -83,3 +83,41 @@ def output_tol(y_ref):
     """Output tolerance: |y - y_ref| <= 2^-7 |y_ref| + 1e-3 max_n |y_ref[m, :]|."""
     y_ref = np.asarray(y_ref, dtype=np.float64)
     return 2.0 ** -7 * np.abs(y_ref) + 1e-3 * np.max(np.abs(y_ref), axis=1, keepdims=True)
+
+
+def check_w4_clip(wr, s_gpu, amax, best_err, ratio, grid):
+    """The GPU's int4 clip choice for one row, checked against the float64
+    clip search ("MossInt4", "Format": per-row clip search over a grid of
+    clip factors, minimum row error).
+
+    The GPU's scale must sit on the clip grid (within its fp32 error), and the
+    float64 row error at that clip must be within the fp32 evaluation error of
+    the float64 optimum `best_err`: the GPU evaluates every candidate in fp32,
+    so two candidates closer than that bound are both acceptable choices.
+    Returns (s64, q): the float64 scale of the chosen grid point and the
+    oracle's codes at that scale, which the caller compares code by code.
+    """
+    wr = np.asarray(wr, dtype=np.float64)
+    c_g = s_gpu * 7.0 / amax
+    i_g = int(np.argmin(np.abs(grid - c_g)))
+    assert abs(c_g - grid[i_g]) <= 1.5 * (ratio + 6 * U) * grid[i_g], "s_row off the clip grid"
+    s64 = grid[i_g] * amax / 7.0
+    q = np.clip(np.rint(wr / s64), -7, 7)
+    err_g = np.sum((wr - s64 * q) ** 2)
+    v2 = np.linalg.norm(wr)
+    # error of one fp32 candidate evaluation: the rotated row (10u ||v||), the
+    # reconstruction s q (its scale's relative error) and the sum of squares
+    dd = 10 * U * v2 + np.linalg.norm(q) * s64 * (ratio + 3 * U) + 2 * U * v2
+    tol_sse = 2 * (2 * np.sqrt(best_err + err_g) * dd + 2 * dd * dd + 48 * U * err_g)
+    # codes inside the tie window may round either way on the GPU
+    win4 = int4_code_window(ratio)
+    z = wr / s64
+    near = np.abs(np.abs(z) - np.floor(np.abs(z)) - 0.5) <= win4
+    tol_sse += near.sum() * 2 * win4 * s64 * s64
+    assert err_g <= best_err + tol_sse, f"clip {grid[i_g]}: row error {err_g} vs best {best_err}"
+    return s64, q
+
+
+def int4_code_window(ratio):
+    """Half-width of the window around a tie in which an int4 code may flip."""
+    return 1.5 * 8.75 * (2.0 * ratio + 4.0 * U)

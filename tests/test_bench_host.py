@@ -23,17 +23,20 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_traffic_only_for_matching_sources(monkeypatch):
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         t = json.load(f)
-    entry = t["down_proj_m512"]["gemm"]
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: entry["source_sha"])
-    assert bench.profiled_traffic("gemm", "down_proj_m512") == entry["dram_bytes_per_launch"]
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)
-    assert bench.profiled_traffic("gemm", "down_proj_m512") is None
+    wl, kernels = next(iter(t.items()))
+    kernel, entry = next(iter(kernels.items()))
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda k: entry["source_sha"])
+    assert bench.profiled_traffic(kernel, wl) == entry["dram_bytes_per_launch"]
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda k: "0" * 16)
+    assert bench.profiled_traffic(kernel, wl) is None
     # an unprofiled kernel or workload has no figure
     assert bench.profiled_traffic("gemm", "no_such_workload") is None
 
 
-def test_source_hash_covers_every_kernel_file(tmp_path, monkeypatch):
-    """The hash changes when any file of the kernel sources changes."""
+@pytest.mark.parametrize("kernel", sorted(bench.KERNEL_SOURCES))
+def test_source_hash_covers_every_file_of_the_kernel(tmp_path, monkeypatch, kernel):
+    """A kernel's hash changes when any file it is built from changes, and
+    only then."""
     src = os.path.join(ROOT, "w8a8_int8_quantized_rmsnorm_b200", "csrc")
     fake = tmp_path / "w8a8_int8_quantized_rmsnorm_b200" / "csrc"
     fake.mkdir(parents=True)
@@ -41,10 +44,21 @@ def test_source_hash_covers_every_kernel_file(tmp_path, monkeypatch):
         with open(os.path.join(src, name), "rb") as f:
             (fake / name).write_bytes(f.read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    h0 = bench.kernel_source_sha()
-    first = sorted(os.listdir(fake))[0]
-    (fake / first).write_bytes((fake / first).read_bytes() + b"\n")
-    assert bench.kernel_source_sha() != h0
+    h0 = bench.kernel_source_sha(kernel)
+    for name in sorted(os.listdir(fake)):
+        before = (fake / name).read_bytes()
+        (fake / name).write_bytes(before + b"\n")
+        changed = bench.kernel_source_sha(kernel) != h0
+        assert changed == (name in bench.KERNEL_SOURCES[kernel]), name
+        (fake / name).write_bytes(before)
+    assert bench.kernel_source_sha(kernel) == h0
+
+
+def test_replay_count_bounds():
+    # one rank: enough replays for MIN_TIMED_MS, within the bounds
+    assert bench.agreed_replays(1000.0, 1, "cpu") == bench.MIN_REPLAYS
+    assert bench.agreed_replays(bench.MIN_TIMED_MS / 20, 1, "cpu") == 20
+    assert bench.agreed_replays(1e-6, 1, "cpu") == bench.MAX_REPLAYS
 
 
 def _commands(text):

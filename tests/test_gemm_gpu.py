@@ -55,6 +55,26 @@ def test_int8_gemm_s32_bit_exact(cr, M, N, K):
     assert np.array_equal(got, want), f"{np.count_nonzero(got != want)} mismatches"
 
 
+def test_int8_gemm_s32_bit_exact_gate_up_m8192(cr):
+    """Every int32 accumulator of the largest single-GPU W8A8 shape (fused
+    gate+up, 8192 tokens x 24576 rows x K 4096: the bench's default
+    workload, in the launch configuration it times) against the oracle's
+    exact integer matmul, in blocks of 1024 tokens."""
+    M, N, K = 8192, 24576, 4096
+    X = _rand_i8((M, K), 8192 + K, -127, 128)
+    W = _rand_i8((N, K), N + K, -127, 128)
+    acc = cr.convrot_int8_gemm_s32(X.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    assert cr.convrot_device_status() == 0
+    got = acc.cpu().numpy()
+    del acc
+    Xn, Wn = X.numpy(), W.numpy()
+    for m0 in range(0, M, 1024):
+        want = ref.int_matmul(Xn[m0:m0 + 1024], Wn)
+        bad = np.count_nonzero(got[m0:m0 + 1024].astype(np.int64) != want)
+        assert bad == 0, f"tokens {m0}..{m0 + 1023}: {bad} mismatches"
+
+
 def test_int8_gemm_s32_extreme_operands(cr):
     M, N, K = 130, 264, 12288
     X = torch.full((M, K), 127, dtype=torch.int8)

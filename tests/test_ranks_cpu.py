@@ -2,7 +2,8 @@
 launches them.  Each GPU rank runs an independent replica (the linear has no
 exchange step), so what the ranks share is the timing: the job's time is the
 slowest rank's (max over ranks) and its throughput is the units all ranks
-processed over that time.  The reference arm runs on rank 0 only."""
+processed over that time, and every rank replays the timed region the same
+number of times.  The reference arm runs on rank 0 only."""
 import os
 import socket
 
@@ -31,6 +32,8 @@ def _rank(rank, world, port, q):
         # entry, rank 0 in the second
         mine = [10.0 + 5.0 * rank, 7.0 - 2.0 * rank]
         got = bench.max_over_ranks(mine, world, "cpu")
+        # the replay count follows the slowest rank's first replay
+        reps = bench.agreed_replays(bench.MIN_TIMED_MS / (10.0 + 10.0 * rank), world, "cpu")
         torch.distributed.barrier()
 
         class A:
@@ -39,7 +42,7 @@ def _rank(rank, world, port, q):
             warmup = 1
 
         ref = bench.run_reference(A, rank, world) if rank != 0 else "rank 0 not run here"
-        q.put((rank, got, ref))
+        q.put((rank, got, ref, reps))
     finally:
         torch.distributed.destroy_process_group()
 
@@ -53,8 +56,8 @@ def test_two_gloo_ranks_max_time_and_reference_rank():
         p.start()
     out = {}
     for _ in procs:
-        rank, got, ref = q.get(timeout=120)
-        out[rank] = (got, ref)
+        rank, got, ref, reps = q.get(timeout=120)
+        out[rank] = (got, ref, reps)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -62,6 +65,9 @@ def test_two_gloo_ranks_max_time_and_reference_rank():
     assert out[0][0] == out[1][0] == [15.0, 7.0]
     # the reference arm does no work on the other ranks
     assert out[1][1] is None
+    # both ranks replay the timed region equally often: enough for the slower
+    # rank (first replay MIN_TIMED_MS / 10 on rank 0, MIN_TIMED_MS / 20 on rank 1)
+    assert out[0][2] == out[1][2] == 10
 
 
 def test_job_throughput_is_all_ranks_units_over_max_time():

@@ -193,23 +193,10 @@ def _w4_check(cr, W, group=256, cs=None, clip=(0.80, 1.00, 21)):
         if amax[n] == 0:
             assert sg[n] == 0 and not codes_gpu[n].any()
             continue
-        c_g = sg[n] * 7.0 / amax[n]
-        i_g = int(np.argmin(np.abs(grid - c_g)))
-        assert abs(c_g - grid[i_g]) <= 1.5 * (ratio[n] + 6 * _tol.U) * grid[i_g], "s_row off the clip grid"
-        s64 = grid[i_g] * amax[n] / 7.0
-        q = np.clip(np.rint(Wr[n] / s64), -7, 7)
-        err_g = np.sum((Wr[n] - s64 * q) ** 2)
-        # the GPU evaluates every candidate's error in fp32; its choice must be
-        # within that evaluation error of the float64 optimum
-        v2 = np.linalg.norm(Wr[n])
-        dd = 10 * _tol.U * v2 + np.linalg.norm(q) * s64 * (ratio[n] + 3 * _tol.U) + 2 * _tol.U * v2
-        tol_sse = 2 * (2 * np.sqrt(out["err"][n] + err_g) * dd + 2 * dd * dd + 48 * _tol.U * err_g)
-        z = Wr[n] / s64
-        win4 = 1.5 * 8.75 * (2 * ratio[n] + 4 * _tol.U)
-        near = np.abs(np.abs(z) - np.floor(np.abs(z)) - 0.5) <= win4
-        tol_sse += near.sum() * 2 * win4 * s64 * s64
-        assert err_g <= out["err"][n] + tol_sse, f"row {n}: clip {grid[i_g]} err {err_g} vs best {out['err'][n]}"
-        _tol.check_codes(codes_gpu[n:n + 1], q[None, :], z[None, :], np.array([win4]), "int4 codes")
+        s64, q = _tol.check_w4_clip(Wr[n], sg[n], amax[n], out["err"][n], ratio[n], grid)
+        win4 = _tol.int4_code_window(ratio[n])
+        _tol.check_codes(codes_gpu[n:n + 1], q[None, :], (Wr[n] / s64)[None, :], np.array([win4]),
+                         "int4 codes")
 
 
 @pytest.mark.parametrize("N,K", [(8, 256), (40, 512), (64, 4096), (16, 12288), (8, 16640)])

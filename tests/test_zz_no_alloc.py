@@ -1,13 +1,15 @@
 """The allocation-free W8A8 linear (convrot_int8_linear_noalloc) against the
-regular entry point (convrot_int8_linear with a caller workspace).
+regular entry point (convrot_int8_linear with a caller workspace) and the
+oracle.
 
 The allocation-free entry point exists for callers that cannot allocate
 device memory where they run the layer; it uses a fixed 24 MiB array inside
 the library as the GEMM's split-tile workspace.  Both entry points run the
 same kernels and schedule, so their outputs must agree within the output
-tolerance the other tests use (in fact bit for bit).  Two calls in a row
-check that the shared array is left fit for the next call.  This file is
-collected last so that, run after the other tests, it also sees a library
+tolerance the other tests use (in fact bit for bit), and both must be within
+one bf16 step of the oracle's correctly rounded float64 result.  Two calls in
+a row check that the shared array is left fit for the next call.  This file
+is collected last so that, run after the other tests, it also sees a library
 that has already served other shapes.
 """
 import ctypes
@@ -16,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import convrot_ref as ref
 from tests import _tol
 
 pytestmark = pytest.mark.gpu
@@ -59,8 +62,13 @@ def test_noalloc_matches_workspace_entry_point_twice(cr, M, N, K):
     X, st, W, sr = _operands(M, N, K, M + N + K)
     want = cr.convrot_int8_linear(X, st, W, sr, workspace=cr.Workspace())
     torch.cuda.synchronize()
-    ref = want.float().cpu().double().numpy()
-    tol = _tol.output_tol(ref)
+    expect = want.float().cpu().double().numpy()
+    tol = _tol.output_tol(expect)
+    # the oracle on the same int8 operands and scales: one bf16 rounding of
+    # the exact float64 dequantisation
+    yb, y64, _ = ref.int8_linear(X.cpu().numpy(), st.cpu().double().numpy(), W.cpu().numpy(),
+                                 sr.cpu().double().numpy())
+    ulp = _tol.bf16_ulp(y64) * 1.0001
     for _ in range(2):
         status, Y = _noalloc_c_abi(cr, X, st, W, sr)
         torch.cuda.synchronize()
@@ -69,8 +77,9 @@ def test_noalloc_matches_workspace_entry_point_twice(cr, M, N, K):
             continue
         assert status == 0
         got = Y.float().cpu().double().numpy()
-        assert np.all(np.abs(got - ref) <= tol)
-        assert np.array_equal(got, ref)
+        assert np.all(np.abs(got - expect) <= tol)
+        assert np.array_equal(got, expect)
+        assert np.all(np.abs(got - yb) <= ulp)
     assert cr.convrot_device_status() == 0
 
 

@@ -51,28 +51,68 @@ def _stream(device: torch.device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def _need(t: torch.Tensor, dtype, name: str, dim: Optional[int] = None):
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (no CPU fallback)")
+def _need(t: torch.Tensor, dtype, name: str, dim: Optional[int] = None, shape=None):
+    """dtype, contiguity and shape of one operand.  The device is checked
+    afterwards, for all operands of a call together (_on_device)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dim is not None and t.dim() != dim:
         raise ValueError(f"{name} must have {dim} dimensions")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _on_device(**operands) -> torch.device:
+    """Every operand is a CUDA tensor on one device, and that device is the
+    current one: the library launches on the current device, on that device's
+    current stream.  None entries (optional operands) are skipped."""
+    dev = None
+    for name, t in operands.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (no CPU fallback)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}; the other operands are on {dev}")
+    cur = torch.cuda.current_device()
+    if dev.index != cur:
+        raise ValueError(f"the operands are on {dev} but the current device is cuda:{cur}")
+    return dev
 
 
 def convrot_version() -> int:
     return lib().convrot_version()
 
 
+# Device timeouts reported so far.  A kernel that gave up on a bounded wait may
+# leave partial sums and tile counters in its split-tile workspace; every
+# Workspace zero-fills itself again before its next use once this has moved.
+_timeouts_reported = 0
+
+
+def _note_status(st: int) -> None:
+    global _timeouts_reported
+    if st == 6:  # CONVROT_ERR_DEVICE_TIMEOUT
+        _timeouts_reported += 1
+
+
 def convrot_device_status(device=None) -> int:
-    """Synchronises the current stream and returns/clears the device error word."""
+    """Synchronises the current stream and returns/clears the device error word.
+
+    A non-zero word means a kernel gave up on a bounded wait; every Workspace
+    is then zero-filled again before its next use."""
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
     detail = ctypes.c_uint32(0)
     st = lib().convrot_device_status(_stream(dev), ctypes.byref(detail))
     if st not in (0, 6):
         _check("convrot_device_status", st)
+    _note_status(st)
     return int(detail.value)
 
 
@@ -80,9 +120,10 @@ def convrot_device_status(device=None) -> int:
 def convrot_quantize_weight(W: torch.Tensor, group: int = 256,
                             col_scale: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     _need(W, torch.bfloat16, "W", 2)
-    if col_scale is not None:
-        _need(col_scale, torch.float32, "col_scale", 1)
     N, K = W.shape
+    if col_scale is not None:
+        _need(col_scale, torch.float32, "col_scale", shape=(K,))
+    _on_device(W=W, col_scale=col_scale)
     Wq = torch.empty(N, K, dtype=torch.int8, device=W.device)
     s_row = torch.empty(N, dtype=torch.float32, device=W.device)
     _check("convrot_quantize_weight", lib().convrot_quantize_weight(
@@ -94,9 +135,10 @@ def convrot_quantize_weight_w4(W: torch.Tensor, group: int = 256,
                                col_scale: Optional[torch.Tensor] = None, clip_lo: float = 0.80,
                                clip_hi: float = 1.00, clip_steps: int = 21):
     _need(W, torch.bfloat16, "W", 2)
-    if col_scale is not None:
-        _need(col_scale, torch.float32, "col_scale", 1)
     N, K = W.shape
+    if col_scale is not None:
+        _need(col_scale, torch.float32, "col_scale", shape=(K,))
+    _on_device(W=W, col_scale=col_scale)
     Wq4 = torch.empty(N, K // 2, dtype=torch.uint8, device=W.device)
     s_row = torch.empty(N, dtype=torch.float32, device=W.device)
     _check("convrot_quantize_weight_w4", lib().convrot_quantize_weight_w4(
@@ -110,11 +152,14 @@ def convrot_smoothquant_calibrate(x: torch.Tensor, norm_w: Optional[torch.Tensor
     """SmoothQuant scales of the linear W fed by x (norm_w None: x reaches W as
     it is, and the second result is scratch)."""
     _need(x, torch.bfloat16, "x", 2)
-    _need(W, torch.bfloat16, "W", 2)
-    if norm_w is not None:
-        _need(norm_w, torch.float32, "norm_w", 1)
     M, K = x.shape
+    _need(W, torch.bfloat16, "W", 2)
     N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("x and W disagree on K")
+    if norm_w is not None:
+        _need(norm_w, torch.float32, "norm_w", shape=(K,))
+    _on_device(x=x, W=W, norm_w=norm_w)
     smooth = torch.empty(K, dtype=torch.float32, device=x.device)
     folded = torch.empty(K, dtype=torch.float32, device=x.device)
     _check("convrot_smoothquant_calibrate", lib().convrot_smoothquant_calibrate(
@@ -128,14 +173,19 @@ def convrot_rotate_quant_act(x: torch.Tensor, group: int = 256,
                              norm_w: Optional[torch.Tensor] = None, eps: float = 1e-6,
                              out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
     _need(x, torch.bfloat16, "x", 2)
-    if norm_w is not None:
-        _need(norm_w, torch.float32, "norm_w", 1)
     M, K = x.shape
+    if norm_w is not None:
+        _need(norm_w, torch.float32, "norm_w", shape=(K,))
+    if out is None:
+        Xq = s_tok = None
+    else:
+        Xq, s_tok = out
+        _need(Xq, torch.int8, "Xq", shape=(M, K))
+        _need(s_tok, torch.float32, "s_tok", shape=(M,))
+    _on_device(x=x, norm_w=norm_w, Xq=Xq, s_tok=s_tok)
     if out is None:
         Xq = torch.empty(M, K, dtype=torch.int8, device=x.device)
         s_tok = torch.empty(M, dtype=torch.float32, device=x.device)
-    else:
-        Xq, s_tok = out
     _check("convrot_rotate_quant_act", lib().convrot_rotate_quant_act(
         _ptr(x), M, K, group, _ptr(norm_w), eps, _ptr(Xq), _ptr(s_tok), _stream(x.device)))
     return Xq, s_tok
@@ -149,20 +199,28 @@ def convrot_linear_workspace_bytes(M: int, N: int, K: int, weight_bits: int = 8)
 class Workspace:
     """Device workspace for the GEMM's split tiles, grown on demand.
 
-    It starts zero-filled; the library keeps its tile counters at zero after
-    every successful call, so it is reused without clearing.  One Workspace
-    must not be used by calls that run concurrently on different streams.
+    It starts zero-filled; the library leaves it zero after every call whose
+    kernels complete, so it is reused without clearing.  After
+    convrot_device_status has reported a device timeout (an aborted call may
+    leave partial sums behind) it is zero-filled again before its next use.
+    One Workspace must not be used by calls that run concurrently on
+    different streams.
     """
 
     def __init__(self, device=None):
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None else device)
         self.buf: Optional[torch.Tensor] = None
+        self.epoch = _timeouts_reported
 
     def get(self, nbytes: int) -> Tuple[Optional[int], int]:
         if nbytes == 0:
             return None, 0
         if self.buf is None or self.buf.numel() < nbytes:
             self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+            self.epoch = _timeouts_reported
+        elif self.epoch != _timeouts_reported:
+            self.buf.zero_()
+            self.epoch = _timeouts_reported
         return self.buf.data_ptr(), self.buf.numel()
 
 
@@ -189,11 +247,22 @@ def _gemm_check(Xq, Wq, w4: bool):
     return M, N, K
 
 
+def _linear_operands(Xq, s_tok, Wq, s_row, out, w4: bool, out_cols=None):
+    """Checks the operands of a W8A8 / W4A8 linear; returns (M, N, K, Y) with
+    Y the caller's `out` or a new bf16 [M, out_cols] tensor."""
+    M, N, K = _gemm_check(Xq, Wq, w4)
+    cols = N if out_cols is None else out_cols
+    _need(s_tok, torch.float32, "s_tok", shape=(M,))
+    _need(s_row, torch.float32, "s_row", shape=(N,))
+    if out is not None:
+        _need(out, torch.bfloat16, "out", shape=(M, cols))
+    dev = _on_device(Xq=Xq, s_tok=s_tok, Wq=Wq, s_row=s_row, out=out)
+    Y = torch.empty(M, cols, dtype=torch.bfloat16, device=dev) if out is None else out
+    return M, N, K, Y
+
+
 def convrot_int8_linear(Xq, s_tok, Wq, s_row, out=None, workspace: Optional[Workspace] = None):
-    M, N, K = _gemm_check(Xq, Wq, False)
-    _need(s_tok, torch.float32, "s_tok", 1)
-    _need(s_row, torch.float32, "s_row", 1)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    M, N, K, Y = _linear_operands(Xq, s_tok, Wq, s_row, out, False)
     ws, wn = _workspace(Xq.device, convrot_linear_workspace_bytes(M, N, K, 8), workspace)
     _check("convrot_int8_linear", lib().convrot_int8_linear(
         _ptr(Xq), _ptr(s_tok), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), ws, wn,
@@ -206,20 +275,14 @@ def convrot_int8_linear_noalloc(Xq, s_tok, Wq, s_row, out=None):
     24 MiB per-device array serves as the split-tile workspace (for callers
     that cannot allocate device memory where they run the layer).  Calls that
     overlap on the GPU race on that array."""
-    M, N, K = _gemm_check(Xq, Wq, False)
-    _need(s_tok, torch.float32, "s_tok", 1)
-    _need(s_row, torch.float32, "s_row", 1)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    M, N, K, Y = _linear_operands(Xq, s_tok, Wq, s_row, out, False)
     _check("convrot_int8_linear_noalloc", lib().convrot_int8_linear_noalloc(
         _ptr(Xq), _ptr(s_tok), _ptr(Wq), _ptr(s_row), M, N, K, _ptr(Y), _stream(Xq.device)))
     return Y
 
 
 def convrot_w4a8_linear(Xq, s_tok, Wq4, s_row, out=None, workspace: Optional[Workspace] = None):
-    M, N, K = _gemm_check(Xq, Wq4, True)
-    _need(s_tok, torch.float32, "s_tok", 1)
-    _need(s_row, torch.float32, "s_row", 1)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    M, N, K, Y = _linear_operands(Xq, s_tok, Wq4, s_row, out, True)
     ws, wn = _workspace(Xq.device, convrot_linear_workspace_bytes(M, N, K, 4), workspace)
     _check("convrot_w4a8_linear", lib().convrot_w4a8_linear(
         _ptr(Xq), _ptr(s_tok), _ptr(Wq4), _ptr(s_row), M, N, K, _ptr(Y), ws, wn,
@@ -229,6 +292,7 @@ def convrot_w4a8_linear(Xq, s_tok, Wq4, s_row, out=None, workspace: Optional[Wor
 
 def convrot_int8_gemm_s32(Xq, Wq, workspace: Optional[Workspace] = None):
     M, N, K = _gemm_check(Xq, Wq, False)
+    _on_device(Xq=Xq, Wq=Wq)
     acc = torch.empty(M, N, dtype=torch.int32, device=Xq.device)
     ws, wn = _workspace(Xq.device, convrot_linear_workspace_bytes(M, N, K, 8), workspace)
     _check("convrot_int8_gemm_s32", lib().convrot_int8_gemm_s32(
@@ -238,6 +302,7 @@ def convrot_int8_gemm_s32(Xq, Wq, workspace: Optional[Workspace] = None):
 
 def convrot_w4a8_gemm_s32(Xq, Wq4, workspace: Optional[Workspace] = None):
     M, N, K = _gemm_check(Xq, Wq4, True)
+    _on_device(Xq=Xq, Wq4=Wq4)
     acc = torch.empty(M, N, dtype=torch.int32, device=Xq.device)
     ws, wn = _workspace(Xq.device, convrot_linear_workspace_bytes(M, N, K, 4), workspace)
     _check("convrot_w4a8_gemm_s32", lib().convrot_w4a8_gemm_s32(
@@ -250,9 +315,12 @@ def convrot_rotate_act_bf16(x: torch.Tensor, group: int = 256, norm_w: Optional[
                             eps: float = 1e-6, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Xr = bf16([RMSNorm] x rotated by the group Hadamard), not quantised."""
     _need(x, torch.bfloat16, "x", 2)
-    if norm_w is not None:
-        _need(norm_w, torch.float32, "norm_w", 1)
     M, K = x.shape
+    if norm_w is not None:
+        _need(norm_w, torch.float32, "norm_w", shape=(K,))
+    if out is not None:
+        _need(out, torch.bfloat16, "out", shape=(M, K))
+    _on_device(x=x, norm_w=norm_w, out=out)
     Xr = torch.empty(M, K, dtype=torch.bfloat16, device=x.device) if out is None else out
     _check("convrot_rotate_act_bf16", lib().convrot_rotate_act_bf16(
         _ptr(x), M, K, group, _ptr(norm_w), eps, _ptr(Xr), _stream(x.device)))
@@ -274,7 +342,10 @@ def convrot_weight_only_workspace_bytes(M: int, N: int, K: int) -> int:
 def convrot_weight_only_linear(Xr, Wq, s_row, out=None, workspace: Optional[Workspace] = None):
     """Y = bf16(s_row * (Xr @ Wq^T)) on rotated bf16 activations, int8 weights."""
     M, N, K = _wo_check(Xr, Wq)
-    _need(s_row, torch.float32, "s_row", 1)
+    _need(s_row, torch.float32, "s_row", shape=(N,))
+    if out is not None:
+        _need(out, torch.bfloat16, "out", shape=(M, N))
+    _on_device(Xr=Xr, Wq=Wq, s_row=s_row, out=out)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xr.device) if out is None else out
     ws, wn = _workspace(Xr.device, convrot_weight_only_workspace_bytes(M, N, K), workspace)
     _check("convrot_weight_only_linear", lib().convrot_weight_only_linear(
@@ -284,6 +355,7 @@ def convrot_weight_only_linear(Xr, Wq, s_row, out=None, workspace: Optional[Work
 
 def convrot_weight_only_gemm_f32(Xr, Wq, workspace: Optional[Workspace] = None):
     M, N, K = _wo_check(Xr, Wq)
+    _on_device(Xr=Xr, Wq=Wq)
     acc = torch.empty(M, N, dtype=torch.float32, device=Xr.device)
     ws, wn = _workspace(Xr.device, convrot_weight_only_workspace_bytes(M, N, K), workspace)
     _check("convrot_weight_only_gemm_f32", lib().convrot_weight_only_gemm_f32(
@@ -298,12 +370,10 @@ def convrot_swiglu_workspace_bytes(M: int, I: int, K: int, weight_bits: int = 8)
 
 def _swiglu(fn, Xq, s_tok, Wq_gu, s_row_gu, w4, out, workspace):
     M, N2, K = _gemm_check(Xq, Wq_gu, w4)
-    _need(s_tok, torch.float32, "s_tok", 1)
-    _need(s_row_gu, torch.float32, "s_row_gu", 1)
     if N2 % 2:
         raise ValueError("the gate/up weight must have an even number of rows")
     I = N2 // 2
-    H = torch.empty(M, I, dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    M, N2, K, H = _linear_operands(Xq, s_tok, Wq_gu, s_row_gu, out, w4, out_cols=I)
     ws, wn = _workspace(Xq.device, convrot_swiglu_workspace_bytes(M, I, K, 4 if w4 else 8), workspace)
     _check(fn, getattr(lib(), fn)(
         _ptr(Xq), _ptr(s_tok), _ptr(Wq_gu), _ptr(s_row_gu), M, I, K, _ptr(H), ws, wn,
@@ -326,8 +396,9 @@ def convrot_interleave_gate_up(Wg: torch.Tensor, Wu: torch.Tensor) -> torch.Tens
     """Rows of gate and up in alternating blocks of 16 (any dtype, 1-D or 2-D)."""
     if Wg.shape != Wu.shape or Wg.dtype != Wu.dtype or Wg.device != Wu.device:
         raise ValueError("gate and up must match in shape, dtype and device")
-    if not (Wg.is_cuda and Wg.is_contiguous() and Wu.is_contiguous()):
-        raise ValueError("gate and up must be contiguous CUDA tensors")
+    if not (Wg.is_contiguous() and Wu.is_contiguous()):
+        raise ValueError("gate and up must be contiguous")
+    _on_device(Wg=Wg, Wu=Wu)
     I = Wg.shape[0]
     row_bytes = Wg.numel() // max(I, 1) * Wg.element_size()
     out = torch.empty((2 * I,) + tuple(Wg.shape[1:]), dtype=Wg.dtype, device=Wg.device)
@@ -339,9 +410,8 @@ def convrot_interleave_gate_up(Wg: torch.Tensor, Wu: torch.Tensor) -> torch.Tens
 def convrot_fold_row_scales(s_row: torch.Tensor, smooth: torch.Tensor) -> torch.Tensor:
     """s_row /= smooth in place (a SmoothQuant scale folded into weight rows)."""
     _need(s_row, torch.float32, "s_row", 1)
-    _need(smooth, torch.float32, "smooth", 1)
-    if s_row.shape != smooth.shape:
-        raise ValueError("s_row and smooth must have the same length")
+    _need(smooth, torch.float32, "smooth", shape=tuple(s_row.shape))
+    _on_device(s_row=s_row, smooth=smooth)
     _check("convrot_fold_row_scales", lib().convrot_fold_row_scales(
         _ptr(s_row), _ptr(smooth), s_row.numel(), _stream(s_row.device)))
     return s_row

@@ -131,6 +131,12 @@ convrot_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
 
+// Number of device timeouts convrot_device_status has reported.  A kernel that
+// gave up on a bounded wait may have left partial sums and tile counters in
+// its split-tile workspace; the library's own fixed workspace is cleared again
+// before its next use when this count has moved.
+std::atomic<unsigned> g_timeouts_reported{0};
+
 // ------------------------------------------------------------------ rowquant
 struct RowPlan {
   int team, rows_per_cta, passes;
@@ -492,13 +498,13 @@ convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const
   stages = std::max(2, stages);
   a.stages = stages;
   const int smem = std::max(SM::total(stages) + 1024, 116 * 1024);
-  static int configured_device_mask = 0;  // per instantiation
+  static std::atomic<bool> configured[64];  // per instantiation and device
   const DeviceInfo d = current_device();
-  const int bit = 1 << (d.device & 31);
-  if (!(configured_device_mask & bit)) {
+  if (d.device < 0) return CONVROT_ERR_CUDA;
+  if (!configured[d.device].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return CONVROT_ERR_CUDA;
-    configured_device_mask |= bit;
+    configured[d.device].store(true, std::memory_order_release);
   }
   constexpr int threads = (W4 || WBF) ? 320 : 192;
   return launch_pdl(k, dim3(grid), dim3(threads), smem, st, 1, ma, mb, my, a);
@@ -720,6 +726,7 @@ convrot_status convrot_device_status(convrot_stream_t stream, uint32_t* detail) 
   if (v && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return CONVROT_ERR_CUDA;
   if (detail) *detail = v;
+  if (v) g_timeouts_reported.fetch_add(1u, std::memory_order_relaxed);
   return v ? CONVROT_ERR_DEVICE_TIMEOUT : CONVROT_OK;
 }
 
@@ -1060,9 +1067,13 @@ convrot_status convrot_w4a8_gemm_s32(const int8_t* Xq, const uint8_t* Wq4, int M
 // the device address is looked up with cudaGetSymbolAddress once per device
 // (the first call on a device does that set-up; make that first call before
 // any stream capture).  All calls on a device share the array and it keeps the
-// last call's contents: each call clears the counters and accumulators it
-// uses, which must start at zero, and calls that overlap on the GPU (other
-// streams, other threads) race on it.
+// last call's contents.  The split-tile counters and accumulators must start
+// at zero: the set-up clears the whole array, every call that completes
+// leaves what it used zero again (the unit that finalises a split tile
+// re-zeroes its accumulator and counter), and after convrot_device_status has
+// reported a device timeout (an aborted call may leave partial sums behind)
+// the next call clears the array again before use.  Calls that overlap on
+// the GPU (other streams, other threads) race on it.
 // ===========================================================================
 constexpr size_t kStaticWorkspaceBytes = static_cast<size_t>(24) << 20;  // 24 MiB per device
 static __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
@@ -1070,15 +1081,25 @@ static __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceByte
 namespace {
 std::mutex g_static_ws_mu;
 void* g_static_ws_ptr[64] = {nullptr};
+// 1 + g_timeouts_reported at the array's last clear on each device (0: never)
+unsigned g_static_ws_clean_at[64] = {0};
 
-// Device address of g_static_workspace on `device` (the current device).
-convrot_status static_workspace_address(int device, void** out) {
+// Device address of g_static_workspace on `device` (the current device),
+// cleared on `stream` if it has not been cleared since set-up or since the
+// last reported device timeout.
+convrot_status static_workspace(int device, cudaStream_t stream, void** out) {
   std::lock_guard<std::mutex> g(g_static_ws_mu);
   if (g_static_ws_ptr[device] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
       return CONVROT_ERR_CUDA;
     g_static_ws_ptr[device] = p;
+  }
+  const unsigned epoch = 1u + g_timeouts_reported.load(std::memory_order_relaxed);
+  if (g_static_ws_clean_at[device] != epoch) {
+    if (cudaMemsetAsync(g_static_ws_ptr[device], 0, kStaticWorkspaceBytes, stream) != cudaSuccess)
+      return CONVROT_ERR_CUDA;
+    g_static_ws_clean_at[device] = epoch;
   }
   *out = g_static_ws_ptr[device];
   return CONVROT_OK;
@@ -1102,10 +1123,8 @@ extern "C" convrot_status convrot_int8_linear_noalloc(const int8_t* Xq, const fl
   if (need > kStaticWorkspaceBytes) return CONVROT_ERR_WORKSPACE;  // shape too large for the array
   void* ws = nullptr;
   if (need > 0) {
-    const convrot_status a = static_workspace_address(d.device, &ws);
+    const convrot_status a = static_workspace(d.device, as_cuda(stream), &ws);
     if (a != CONVROT_OK) return a;
-    // the counters and accumulators this call uses must start at zero
-    if (cudaMemsetAsync(ws, 0, need, as_cuda(stream)) != cudaSuccess) return CONVROT_ERR_CUDA;
   }
   return run_gemm(Xq, Wq, false, s_tok, s_row, M, N, K, Y, EPI_BF16, ws,
                   need > 0 ? kStaticWorkspaceBytes : 0, as_cuda(stream));
