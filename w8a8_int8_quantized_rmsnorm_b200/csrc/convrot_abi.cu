@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "../../include/convrot.h"
+#include "actquant.cuh"
 #include "gemm.cuh"
 #include "gemm2sm.cuh"
 #include "rowquant.cuh"
@@ -127,6 +128,69 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row
                   box_bytes, swizzle128);
 }
 
+// An N-d tiled map (N <= 3) of elements of `esize` bytes with the given
+// dimensions (innermost first), byte strides of dimensions 1..N-1, box and
+// swizzle; cached per thread like make_map.
+bool make_map_nd(CUtensorMap* map, const void* base, int rank, CUtensorMapDataType dtype,
+                 int esize, const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
+                 bool swizzle128) {
+  struct Key {
+    const void* base;
+    int rank, dtype, esize, swz;
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    bool operator==(const Key& o) const {
+      return std::memcmp(this, &o, sizeof(Key)) == 0;
+    }
+  };
+  struct Entry {
+    Key key;
+    CUtensorMap map;
+    bool valid;
+  };
+  constexpr int kCache = 16;
+  thread_local Entry cache[kCache] = {};
+  thread_local int next = 0;
+  Key key;
+  std::memset(&key, 0, sizeof(key));
+  key.base = base;
+  key.rank = rank;
+  key.dtype = static_cast<int>(dtype);
+  key.esize = esize;
+  key.swz = swizzle128 ? 1 : 0;
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+    if (i + 1 < rank) key.strides[i] = strides[i];
+  }
+  for (int i = 0; i < kCache; ++i) {
+    if (cache[i].valid && cache[i].key == key) {
+      *map = cache[i].map;
+      return true;
+    }
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 1 || rank > 3) return false;
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  const CUresult r = fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st,
+                        bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  Entry& e = cache[next];
+  next = (next + 1) % kCache;
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
+  return true;
+}
+
 convrot_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? CONVROT_OK : CONVROT_ERR_CUDA;
 }
@@ -230,41 +294,91 @@ convrot_status launch_rowquant_pre(RowQuantArgs& a, int group, cudaStream_t st) 
   return launch_rowquant_grp<0, PRE, QK>(a, p, st);
 }
 
-// TMA-fed activation kernel: teams of rowquant's layout, one CTA per SM, a
-// ring of stages of `rows` token rows each.
-template <int GRP, bool NORM>
-convrot_status launch_actquant_t(ActArgs a, cudaStream_t st) {
-  auto k = actquant_kernel<GRP, NORM>;
+// TMA-fed activation kernel: one CTA per SM, a ring of stages of `rows`
+// token rows each, teams of eight threads per 256-element group.  The rows
+// are staged as [rows][K / 64][64] boxes and the norm weight as [K / 32][32]
+// lines, both with the 128-byte swizzle.
+template <int GRP, bool NORM, bool WIDE>
+convrot_status launch_actquant_w(const ActArgs& a, const float* norm_w, cudaStream_t st) {
+  auto k = actquant_kernel<GRP, NORM, WIDE>;
   const DeviceInfo d = current_device();
-  const int dyn = a.wsm_bytes + a.stages * a.rows * a.K * 2;
-  static std::atomic<int> configured[64];
-  if (d.device >= 0 && configured[d.device].load(std::memory_order_relaxed) < dyn) {
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+  if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
+  CUtensorMap mx, mw;
+  const uint64_t xdims[3] = {64, static_cast<uint64_t>(a.K / 64), static_cast<uint64_t>(a.M)};
+  const uint64_t xstr[2] = {128, static_cast<uint64_t>(a.K) * 2};
+  const uint32_t xbox[3] = {64, static_cast<uint32_t>(a.K / 64), static_cast<uint32_t>(a.group_rows)};
+  if (!make_map_nd(&mx, a.x, 3, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xdims, xstr, xbox, true))
+    return CONVROT_ERR_CUDA;
+  if (NORM) {
+    const uint64_t wdims[2] = {32, static_cast<uint64_t>(a.K / 32)};
+    const uint64_t wstr[1] = {128};
+    const uint32_t wbox[2] = {32, static_cast<uint32_t>(a.w_box_lines)};
+    if (!make_map_nd(&mw, norm_w, 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, wdims, wstr, wbox, true))
+      return CONVROT_ERR_CUDA;
+  } else {
+    std::memset(&mw, 0, sizeof(mw));
+  }
+  const int groups = a.rows / a.group_rows;
+  const int dyn = 1024 + a.wsm_bytes + a.xpose_bytes + groups * a.stages * a.slot_stride;
+  static std::atomic<bool> configured[64];
+  if (!configured[d.device].load(std::memory_order_acquire)) {
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AQ_SMEM_BUDGET) !=
         cudaSuccess)
       return CONVROT_ERR_CUDA;
-    configured[d.device].store(200 * 1024, std::memory_order_relaxed);
+    configured[d.device].store(true, std::memory_order_release);
   }
   const int units = (a.M + a.rows - 1) / a.rows;
-  const int grid = std::max(1, std::min(units, std::max(1, d.sms)));
-  return launch_pdl(k, dim3(grid), dim3(32 + a.team * a.rows), dyn, st, 1, a);
+  const int grid = std::max(1, std::min(units, d.sms));
+  return launch_pdl(k, dim3(grid), dim3(a.team * a.rows), dyn, st, 1, mx, mw, a);
 }
 
-// Returns false when the shape is outside what the TMA-fed kernel handles
-// (rows wider than one team of 256 threads), so the caller uses rowquant_kernel.
-bool plan_actquant(int K, ActArgs& a) {
-  const RowPlan p = plan_rows(K);
-  if (!p.resident) return false;
-  a.team = p.team;
-  // up to 12 consumer warps: several rows in flight per CTA
-  a.rows = std::max(1, 384 / p.team);
-  const int row_bytes = K * 2;
-  // keep a stage within 48 KB
-  while (a.rows > 1 && a.rows * row_bytes > 48 * 1024) --a.rows;
-  if (a.team * a.rows < 32 || (a.team * a.rows) % 32) return false;
-  a.wsm_bytes = 0;
-  const int budget = 200 * 1024;
-  const int stage = a.rows * row_bytes;
-  a.stages = std::min(ACT_MAX_STAGES, budget / stage);
+// teams of whole warps (K >= 1024) reduce with redux and a fixed shuffle tree
+template <int GRP, bool NORM>
+convrot_status launch_actquant_t(const ActArgs& a, const float* norm_w, cudaStream_t st) {
+  return a.team >= 32 ? launch_actquant_w<GRP, NORM, true>(a, norm_w, st)
+                      : launch_actquant_w<GRP, NORM, false>(a, norm_w, st);
+}
+
+// Team and stage plan of the activation kernel: eight threads per (virtual)
+// 256-element group, padded to a power of two below a warp or to whole warps;
+// as many rows per stage as fit in AQ_MAX_CWARPS consumer warps, but no more
+// than needed to give every SM a row first.  Returns false when K is not a
+// multiple of 64 (the staged lines), the row is wider than AQ_MAX_TEAM_WARPS
+// warps or the ring would hold fewer than two stages (the caller then uses
+// rowquant_kernel).
+bool plan_actquant(int M, int K, int group, bool norm, int sms, ActArgs& a) {
+  if (K % 64) return false;
+  const int lanes = 8 * ((K + 255) / 256);
+  int team;
+  if (lanes <= 32) {
+    team = 8;
+    while (team < lanes) team <<= 1;
+  } else {
+    team = (lanes + 31) / 32 * 32;
+  }
+  if (team > 32 * AQ_MAX_TEAM_WARPS) return false;
+  const int team_warps = std::max(1, team / 32);
+  const int max_rows = team >= 32 ? AQ_MAX_CWARPS / team_warps : AQ_MAX_CWARPS * (32 / team);
+  const int per_sm = (M + std::max(1, sms) - 1) / std::max(1, sms);
+  int rows = std::max(1, std::min(max_rows, per_sm));
+  if (team < 32) rows = (rows * team + 31) / 32 * 32 / team;  // whole consumer warps
+  if (team > 32 && rows > AQ_MAX_SLOTS) rows = AQ_MAX_SLOTS;  // one named barrier per row slot
+  if (rows > 256) return false;                               // TMA box dimension
+  const int cwarps = rows * team / 32;
+  a.team = team;
+  a.rows = rows;
+  const int wlines = K / 32;
+  a.w_copies = norm ? (wlines + 255) / 256 : 0;
+  a.w_box_lines = norm ? (wlines + a.w_copies - 1) / a.w_copies : 0;
+  a.wsm_bytes = norm ? (a.w_copies * a.w_box_lines * 128 + 1023) / 1024 * 1024 : 0;
+  a.xpose_bytes = group == 256 ? cwarps * AQ_XPOSE_WARP_BYTES : 0;
+  // staging groups: one per team of whole warps, one per warp of narrow teams
+  a.group_rows = team >= 32 ? 1 : 32 / team;
+  const int groups = rows / a.group_rows;
+  if (groups > AQ_MAX_RINGS) return false;
+  a.slot_stride = (a.group_rows * K * 2 + 1023) / 1024 * 1024;
+  a.stages = std::min(AQ_MAX_STAGES, (AQ_SMEM_BUDGET - 1024 - a.wsm_bytes - a.xpose_bytes) /
+                                         (groups * a.slot_stride));
   return a.stages >= 2;
 }
 
@@ -802,25 +916,23 @@ convrot_status convrot_rotate_quant_act(const void* x, int M, int K, int group,
   if (norm_w && !aligned(norm_w, 16)) return CONVROT_ERR_ALIGN;
   ActArgs q{};
   q.x = static_cast<const uint16_t*>(x);
-  q.norm_w = norm_w;
   q.xq = Xq;
   q.s_tok = s_tok;
   q.M = M;
   q.K = K;
   q.eps = eps;
-  if (plan_actquant(K, q)) {
-    if (norm_w) {
-      q.wsm_bytes = (K * 4 + 1023) / 1024 * 1024;
-      q.stages = std::min(ACT_MAX_STAGES, (200 * 1024 - q.wsm_bytes) / (q.rows * K * 2));
-    }
-    if (q.stages >= 2) {
-      cudaStream_t st = as_cuda(stream);
-      if (group == 256)
-        return norm_w ? launch_actquant_t<256, true>(q, st) : launch_actquant_t<256, false>(q, st);
-      if (group == 16)
-        return norm_w ? launch_actquant_t<16, true>(q, st) : launch_actquant_t<16, false>(q, st);
-      return norm_w ? launch_actquant_t<0, true>(q, st) : launch_actquant_t<0, false>(q, st);
-    }
+  const DeviceInfo d = current_device();
+  if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
+  if (plan_actquant(M, K, group, norm_w != nullptr, d.sms, q)) {
+    cudaStream_t st = as_cuda(stream);
+    if (group == 256)
+      return norm_w ? launch_actquant_t<256, true>(q, norm_w, st)
+                    : launch_actquant_t<256, false>(q, norm_w, st);
+    if (group == 16)
+      return norm_w ? launch_actquant_t<16, true>(q, norm_w, st)
+                    : launch_actquant_t<16, false>(q, norm_w, st);
+    return norm_w ? launch_actquant_t<0, true>(q, norm_w, st)
+                  : launch_actquant_t<0, false>(q, norm_w, st);
   }
   RowQuantArgs a{};
   a.src = static_cast<const uint16_t*>(x);

@@ -73,10 +73,6 @@ constexpr int EPI_S32 = 1;
 constexpr int EPI_SWIGLU = 2;
 constexpr int SWIGLU_BLOCK = 16;
 
-// wait sites recorded in the device error word
-constexpr unsigned SITE_PROD_EMPTY = 1, SITE_MMA_FULL = 2, SITE_MMA_TMEM = 3, SITE_EPI_FULL = 4,
-                   SITE_CONV_FULL = 5, SITE_DRAIN = 6, SITE_EPI_SYNC = 7, SITE_SPLIT = 8;
-
 struct GemmArgs {
   int M, N, K;
   int rowsA, rowsB;  // rows of operands A and B

@@ -23,6 +23,10 @@ constexpr unsigned ERR_BAD_ARGUMENT = 2u;
 // ~1.1 s at 1.9 GHz: far beyond any legitimate wait inside these kernels.
 constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;
 
+// wait sites recorded in the device error word
+constexpr unsigned SITE_PROD_EMPTY = 1, SITE_MMA_FULL = 2, SITE_MMA_TMEM = 3, SITE_EPI_FULL = 4,
+                   SITE_CONV_FULL = 5, SITE_DRAIN = 6, SITE_EPI_SYNC = 7, SITE_SPLIT = 8;
+
 __device__ __forceinline__ void report_error(unsigned bits) { atomicOr(&g_error_word, bits); }
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -100,6 +104,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_limit(bar, parity, abort, site, WAIT_LIMIT_CYCLES);
 }
 
+// The same bounded wait for short, frequent waits: plain try_wait probes (no
+// suspend-time hint), so a waiting thread resumes as soon as the phase
+// completes.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               unsigned site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long start = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (clock64() - start > WAIT_LIMIT_CYCLES) {
+        report_error(ERR_WAIT_TIMEOUT | ((site & 0xFFu) << 8));
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -114,6 +138,27 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1),
       "l"(cache_policy)
+      : "memory");
+}
+
+// 3-D tiled bulk tensor load global -> shared, completing on `bar` (no
+// multicast; c0 innermost, in elements).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// 2-D tiled load without a cache hint.
+__device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                  int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
 
@@ -191,6 +236,19 @@ __device__ __forceinline__ void bulk_wait_group() {
 }
 
 // 16-byte shared-memory load (explicit state space: LDS, short scoreboard).
+// 16-byte shared-memory load / store at a 32-bit shared address.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(a));
+  return r;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(const void* p) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"

@@ -471,366 +471,6 @@ __global__ void __launch_bounds__(256) rowquant_kernel(RowQuantArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Activation rotate-quantise for the per-token hot path, fed by TMA.
-//
-// One CTA per SM.  Warp 0 (one lane) streams "stages" of R consecutive token
-// rows into a ring of shared-memory buffers with 1-D bulk copies (one copy per
-// stage: the rows are contiguous in HBM) and prefetches later stages into L2.
-// The other warps form R teams of T = (padded) K/64 threads; team r takes row r
-// of a stage, reads its 64 elements per thread from shared memory in the same
-// lane layout as rowquant_kernel, releases the stage at once, and runs the
-// 256-point FWHT in packed f32x2 arithmetic (lane bits by shuffles), the row
-// reductions and 8-byte code stores.  The RMSNorm weight w is bulk-copied once
-// per CTA into shared memory together with the first rows.
-// ---------------------------------------------------------------------------
-constexpr int ACT_MAX_STAGES = 8;
-
-struct ActArgs {
-  const uint16_t* x;   // [M, K] bf16 bits
-  const float* norm_w; // [K] or null
-  int8_t* xq;          // [M, K]
-  float* s_tok;        // [M]
-  int M, K;
-  float eps;
-  int team;            // threads per row (as rowquant_kernel)
-  int rows;            // rows per stage (teams per CTA)
-  int stages;
-  int wsm_bytes;       // shared bytes for 1 + w (K * 4 rounded up to 1024, or 0)
-};
-
-__device__ __forceinline__ uint32_t q8_byte(float v, float inv) {
-  // rint(v * inv) in one rounding: adding 1.5 * 2^23 leaves the integer in the
-  // low mantissa bits (round-half-even); its low byte is the two's-complement
-  // int8 code (|v * inv| <= 127 by construction of inv)
-  return __float_as_uint(fmaf(v, inv, 12582912.0f));
-}
-
-__device__ __forceinline__ uint32_t pack4_bytes(uint32_t q0, uint32_t q1, uint32_t q2, uint32_t q3) {
-  return __byte_perm(__byte_perm(q0, q1, 0x0040), __byte_perm(q2, q3, 0x0040), 0x5410);
-}
-
-__device__ __forceinline__ void act_store_int8(int8_t* row, int K, int g, int L, bool ok,
-                                               const float (&v)[64], float inv) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int j = 32 * h + 16 * q + 4 * k;
-        w[k] = pack4_bytes(q8_byte(v[j], inv), q8_byte(v[j + 1], inv), q8_byte(v[j + 2], inv),
-                           q8_byte(v[j + 3], inv));
-      }
-      const int e = g * 256 + 128 * h + 32 * L + 16 * q;
-      if (ok && e < K) st_v4(row + e, make_uint4(w[0], w[1], w[2], w[3]));
-    }
-  }
-}
-
-template <bool NORM>
-__device__ __forceinline__ void act_load_smem(const uint16_t* srow, const float* wsm, int K, int g,
-                                              int L, bool ok, float (&v)[64], float& sq) {
-  float part[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = g * 256 + i * 32 + L * 8;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (ok && e < K) raw = *reinterpret_cast<const uint4*>(srow + e);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      v[8 * i + 2 * h] = __uint_as_float(w[h] << 16);
-      v[8 * i + 2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
-    }
-    float p0 = v[8 * i] * v[8 * i] + v[8 * i + 1] * v[8 * i + 1];
-    float p1 = v[8 * i + 2] * v[8 * i + 2] + v[8 * i + 3] * v[8 * i + 3];
-    float p2 = v[8 * i + 4] * v[8 * i + 4] + v[8 * i + 5] * v[8 * i + 5];
-    float p3 = v[8 * i + 6] * v[8 * i + 6] + v[8 * i + 7] * v[8 * i + 7];
-    part[i] = (p0 + p1) + (p2 + p3);
-    if (NORM) {
-      float4 m0 = make_float4(0.f, 0.f, 0.f, 0.f), m1 = m0;
-      if (ok && e < K) {
-        m0 = *reinterpret_cast<const float4*>(wsm + e);
-        m1 = *reinterpret_cast<const float4*>(wsm + e + 4);
-      }
-      v[8 * i] *= m0.x; v[8 * i + 1] *= m0.y; v[8 * i + 2] *= m0.z; v[8 * i + 3] *= m0.w;
-      v[8 * i + 4] *= m1.x; v[8 * i + 5] *= m1.y; v[8 * i + 6] *= m1.z; v[8 * i + 7] *= m1.w;
-    }
-  }
-  sq += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-}
-
-// Packed fp32x2 arithmetic (one instruction for two lanes of a 64-bit register).
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
-}
-__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
-__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
-
-// Lane (g, L) of a 256-group holds elements 32i + 8L + r (i, r = 0..7) as 32
-// pairs: pair p = 4i + r/2 holds (r even, r odd).  Loads them from a staged
-// row in shared memory, accumulates sum(x^2) and applies the norm multiplier
-// 1 + w (wsm holds w).
-// WHOLE: K is a multiple of 256, so a lane whose group exists is in range.
-template <bool NORM, bool WHOLE>
-__device__ __forceinline__ void act3_load(const uint16_t* srow, const float* wsm, int K, int g,
-                                          int L, bool ok, uint64_t (&v)[32], float& sq) {
-  float part[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = g * 256 + i * 32 + L * 8;
-    const bool in = WHOLE ? ok : (ok && e < K);
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (in) raw = ld_shared_v4(srow + e);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint64_t acc = 0;
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const uint64_t x2 = static_cast<uint64_t>(w[h] << 16) | (static_cast<uint64_t>(w[h] & 0xFFFF0000u) << 32);
-      acc = h == 0 ? f2_mul(x2, x2) : f2_fma(x2, x2, acc);
-      v[4 * i + h] = x2;
-    }
-    part[i] = f2_lo(acc) + f2_hi(acc);
-    if (NORM) {
-      ulonglong2 m0 = make_ulonglong2(0ull, 0ull), m1 = m0;
-      if (in) {
-        const uint4 u0 = ld_shared_v4(wsm + e), u1 = ld_shared_v4(wsm + e + 4);
-        m0 = make_ulonglong2(u0.x | (static_cast<uint64_t>(u0.y) << 32),
-                             u0.z | (static_cast<uint64_t>(u0.w) << 32));
-        m1 = make_ulonglong2(u1.x | (static_cast<uint64_t>(u1.y) << 32),
-                             u1.z | (static_cast<uint64_t>(u1.w) << 32));
-      }
-      // x * (1 + w) as x + x * w: one rounding of the exact product
-      v[4 * i] = f2_fma(v[4 * i], m0.x, v[4 * i]);
-      v[4 * i + 1] = f2_fma(v[4 * i + 1], m0.y, v[4 * i + 1]);
-      v[4 * i + 2] = f2_fma(v[4 * i + 2], m1.x, v[4 * i + 2]);
-      v[4 * i + 3] = f2_fma(v[4 * i + 3], m1.y, v[4 * i + 3]);
-    }
-  }
-  sq += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-}
-
-// Unnormalised FWHT of the GRP-element groups (256 or 16) within the 256
-// elements held by four lanes, in place.
-template <int GRP>
-__device__ __forceinline__ void act3_fwht(uint64_t (&v)[32], int lane) {
-  // element bit 0: inside each pair
-#pragma unroll
-  for (int p = 0; p < 32; ++p) {
-    const float x = f2_lo(v[p]), y = f2_hi(v[p]);
-    v[p] = f2_pack(x + y, x - y);
-  }
-  // element bits 1, 2 (and 5, 6, 7 for 256-point groups): between pairs
-  // (pair-index bits 0..4)
-#pragma unroll
-  for (int m = 1; m < (GRP == 256 ? 32 : 4); m <<= 1) {
-#pragma unroll
-    for (int p = 0; p < 32; ++p) {
-      if (!(p & m)) {
-        const uint64_t x = v[p], y = v[p | m];
-        v[p] = f2_add(x, y);
-        v[p | m] = f2_sub(x, y);
-      }
-    }
-  }
-  // element bits 3 (and 4): between lanes (lane bits 0, 1).  The lane whose
-  // bit is clear keeps x + partner, the other partner - x.
-#pragma unroll
-  for (int lm = 1; lm <= (GRP == 256 ? 2 : 1); lm <<= 1) {
-    const float sg = (lane & lm) ? -1.0f : 1.0f;
-    const uint64_t s2 = f2_pack(sg, sg);
-#pragma unroll
-    for (int p = 0; p < 32; ++p) {
-      const uint32_t lo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v[p]), lm);
-      const uint32_t hi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v[p] >> 32), lm);
-      v[p] = f2_fma(v[p], s2, static_cast<uint64_t>(lo) | (static_cast<uint64_t>(hi) << 32));
-    }
-  }
-}
-
-__device__ __forceinline__ float act3_absmax(const uint64_t (&v)[32]) {
-  float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
-#pragma unroll
-  for (int p = 0; p < 32; p += 2) {
-    m0 = fmaxf(m0, fabsf(f2_lo(v[p])));
-    m1 = fmaxf(m1, fabsf(f2_hi(v[p])));
-    m2 = fmaxf(m2, fabsf(f2_lo(v[p + 1])));
-    m3 = fmaxf(m3, fabsf(f2_hi(v[p + 1])));
-  }
-  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-}
-
-// int8 codes rint(v * inv) (one rounding, half-even), 8 bytes per i.
-template <bool WHOLE>
-__device__ __forceinline__ void act3_store(int8_t* row, int K, int g, int L, bool ok,
-                                           const uint64_t (&v)[32], float inv) {
-  const uint64_t inv2 = f2_pack(inv, inv);
-  const uint64_t mag2 = f2_pack(12582912.0f, 12582912.0f);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint32_t q[8];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const uint64_t t = f2_fma(v[4 * i + h], inv2, mag2);
-      q[2 * h] = static_cast<uint32_t>(t);
-      q[2 * h + 1] = static_cast<uint32_t>(t >> 32);
-    }
-    const uint32_t w0 = pack4_bytes(q[0], q[1], q[2], q[3]);
-    const uint32_t w1 = pack4_bytes(q[4], q[5], q[6], q[7]);
-    const int e = g * 256 + i * 32 + L * 8;
-    if (WHOLE ? ok : (ok && e < K))
-      asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(row + e), "r"(w0), "r"(w1) : "memory");
-  }
-}
-
-template <int GRP, bool NORM>
-__global__ void __launch_bounds__(416, 1) actquant_kernel(ActArgs a) {
-  // K is a multiple of 256 for 256-point groups: no per-element bounds checks
-  constexpr bool WHOLE = GRP == 256;
-  pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
-  __shared__ float s_max[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
-  __shared__ double s_sum[2 * RQ_MAX_SLOTS * RQ_MAX_WARPS_PER_TEAM];
-  __shared__ uint64_t full[ACT_MAX_STAGES], empty[ACT_MAX_STAGES], wbar;
-  __shared__ int abort_word;
-  extern __shared__ __align__(1024) uint8_t act_smem[];
-  float* wsm = reinterpret_cast<float*>(act_smem);
-  uint8_t* ring = act_smem + a.wsm_bytes;
-  const int stage_bytes = a.rows * a.K * 2;
-  volatile int* abort_flag = &abort_word;
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int consumers = a.team * a.rows;
-  const int cwarps = consumers >> 5;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < a.stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], cwarps);
-    }
-    mbar_init(&wbar, 1);
-    abort_word = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  pdl_wait();  // x, w, Xq and s_tok may belong to the previous kernel
-
-  const int units = (a.M + a.rows - 1) / a.rows;
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      if (NORM) {
-        // the norm weight w [K] fp32, copied once per CTA next to the first rows
-        mbar_arrive_expect_tx(&wbar, static_cast<uint32_t>(a.K) * 4u);
-        bulk_load_1d(wsm, a.norm_w, static_cast<uint32_t>(a.K) * 4u, &wbar);
-      }
-      int i = 0;
-      for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
-        const int s = i % a.stages;
-        const uint32_t ph = (i / a.stages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, SITE_PROD_EMPTY)) break;
-        const int r0 = u * a.rows;
-        const int nrows = min(a.rows, a.M - r0);
-        const uint32_t bytes = static_cast<uint32_t>(nrows) * a.K * 2;
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_load_1d(ring + s * stage_bytes, a.x + static_cast<size_t>(r0) * a.K, bytes, &full[s]);
-        // warm L2 with the unit this CTA loads `stages` steps later
-        const int uf = u + a.stages * gridDim.x;
-        if (uf < units) {
-          const int rf = uf * a.rows;
-          bulk_prefetch_l2(a.x + static_cast<size_t>(rf) * a.K,
-                           static_cast<uint32_t>(min(a.rows, a.M - rf)) * a.K * 2);
-        }
-      }
-      // drain: every issued copy has landed (consumers waited on each) unless
-      // a wait gave up; wait (bounded) for the last ones before exiting
-      const int issued = i;
-      for (int j = max(0, issued - a.stages); j < issued; ++j) {
-        int dummy = 0;
-        mbar_wait(&full[j % a.stages], (j / a.stages) & 1u, &dummy, SITE_DRAIN);
-      }
-      if (NORM) {
-        int dummy = 0;
-        mbar_wait(&wbar, 0u, &dummy, SITE_DRAIN);
-      }
-    }
-    return;
-  }
-  // ------------------------------------------------------------ consumers
-  const int ct = threadIdx.x - 32;
-  const int slot = ct / a.team;
-  const int t = ct - slot * a.team;
-  const int L = t & 3;
-  const int g = t >> 2;
-  const int G = (a.K + 255) >> 8;
-  TeamReducer red{s_max, s_sum, a.team, slot, lane, t >> 5, a.team >> 5, 0};
-  if (NORM && !mbar_wait(&wbar, 0u, abort_flag, SITE_EPI_FULL)) return;
-  int i = 0;
-  for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
-    const int s = i % a.stages;
-    const uint32_t ph = (i / a.stages) & 1u;
-    const bool got = mbar_wait(&full[s], ph, abort_flag, SITE_EPI_FULL);
-    // every consumer warp takes the same decision (abort is CTA-wide), so the
-    // team reductions below stay matched
-    if (!got) break;
-    const int row = u * a.rows + slot;
-    const bool row_ok = row < a.M;
-    const uint16_t* srow =
-        reinterpret_cast<const uint16_t*>(ring + s * stage_bytes) + static_cast<size_t>(slot) * a.K;
-    uint64_t v[32];
-    float sq = 0.f;
-    act3_load<NORM, WHOLE>(srow, wsm, a.K, g, L, row_ok && g < G, v, sq);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);  // stage read: the producer may refill it
-    if (GRP) act3_fwht<GRP>(v, lane);
-    float amax = act3_absmax(v);
-    double sumsq = static_cast<double>(sq);
-    red.reduce(amax, sumsq);
-    if (NORM) {
-      const bool need = amax > 0.f && !(sumsq > 0x1p-100 && sumsq < 0x1p+100);
-      if (__any_sync(0xffffffffu, need)) {
-        const uint16_t* grow = a.x + static_cast<size_t>(row_ok ? row : 0) * a.K;
-        RowQuantArgs ra{};
-        ra.K = a.K;
-        double s64 = rq_sumsq64(ra, grow, g, L, row_ok && g < G);
-        float dummy = 0.f;
-        red.reduce(dummy, s64);
-        if (need) sumsq = s64;
-      }
-    }
-    const float inv = amax > 0.f ? 127.0f / amax : 0.0f;
-    if (row_ok && t == 0) {
-      // the per-row scale is needed by one thread only
-      double rowfac = group_norm<GRP>();
-      if (NORM) rowfac *= 1.0 / sqrt(sumsq / static_cast<double>(a.K) + static_cast<double>(a.eps));
-      a.s_tok[row] = amax > 0.f ? static_cast<float>(static_cast<double>(amax) * rowfac / 127.0) : 0.0f;
-    }
-    act3_store<WHOLE>(a.xq + static_cast<size_t>(row_ok ? row : 0) * a.K, a.K, g, L, row_ok && g < G,
-                    v, inv);
-  }
-}
-
-// ---------------------------------------------------------------------------
 // SmoothQuant calibration (offline): column maxima of the normalised
 // activation and of the weight, then s = ax^alpha / aw^(1-alpha).
 // ---------------------------------------------------------------------------
