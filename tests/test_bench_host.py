@@ -104,3 +104,17 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
     assert r["cores"] >= 1
     assert r["single_thread"]["cores"] == 1 and r["single_thread"]["value"] > 0
+
+
+def test_clock_summary_counts_only_the_timed_region():
+    """Samples before and after the timed region (idle clocks) are left out;
+    the throttle reasons are those seen inside it."""
+    def line(mhz, cap):
+        return f"0, {mhz}, 1965, 990.5, 0x4, Not Active, Not Active, Not Active, {cap}"
+    lines = [(0.5, line(1965, "Not Active")), (1.0, line(1440, "Active")),
+             (1.1, line(1425, "Active")), (1.2, line(1455, "Not Active")),
+             (2.5, line(1965, "Not Active")), (3.0, "garbage")]
+    r = bench.summarize_clocks(lines, 0.9, 2.0)
+    assert r["samples"] == 3 and r["sm_mhz"] == 1440.0 and r["sm_min_mhz"] == 1425.0
+    assert r["reasons"] == ["sw_power_cap"] and r["sm_max_mhz"] == 1965.0
+    assert bench.summarize_clocks(lines)["samples"] == 5
