@@ -123,6 +123,19 @@ def test_act_scale_invariance_with_norm(cr):
     assert torch.allclose(s1, s2, rtol=4e-7, atol=0)
 
 
+@pytest.mark.parametrize("M,K,norm", [(5000, 1024, False), (2300, 2048, True), (1203, 4096, True),
+                                      (601, 8192, False), (301, 16384, True), (901, 12288, False)])
+def test_act_full_cta_plans(cr, M, K, norm):
+    # M large enough that every CTA stages its full complement of rows: 32 warps
+    # per CTA for teams of 1, 2, 4, 8 and 16 warps, 24 for the 12-warp team of
+    # K = 12288; M is no multiple of the rows per stage, so the last unit is
+    # ragged; every row checked
+    x = workloads.activations(M, K, outlier_count=max(1, K // 100), seed=M + K)
+    nw = workloads.norm_weight(K) if norm else None
+    flips = _check_act(cr, x, 256, nw)
+    assert flips <= 1e-4 * x.numel()
+
+
 def test_act_full_size_down_proj(cr):
     # the down-proj workload at full size, every row checked
     w = workloads.WORKLOADS["down_proj_m512"]

@@ -52,12 +52,12 @@
 namespace convrot {
 
 constexpr int AQ_MAX_STAGES = 8;
-constexpr int AQ_MAX_CWARPS = 24;      // warps per CTA, all consumers
+constexpr int AQ_MAX_CWARPS = 32;      // warps per CTA, all consumers (24 or 32 per launch)
 constexpr int AQ_MAX_TEAM_WARPS = 16;  // a row of up to 16384 elements
 constexpr int AQ_MAX_SLOTS = 15;       // rows per stage for teams wider than a warp (barriers 1..15)
 constexpr int AQ_XPOSE_WARP_BYTES = 2048;  // exchange halves: four groups x 512 bytes
-constexpr int AQ_SMEM_BUDGET = 216 * 1024;  // dynamic; the static arrays take ~9 KB more
-constexpr int AQ_MAX_RINGS = 24;       // staging groups per CTA (a team, or a warp of narrow teams)
+constexpr int AQ_SMEM_BUDGET = 214 * 1024;  // dynamic; the static arrays take ~11 KB more
+constexpr int AQ_MAX_RINGS = 32;       // staging groups per CTA (a team, or a warp of narrow teams)
 
 struct ActArgs {
   const uint16_t* x;    // [M, K] bf16 bits (L2 prefetch and the rare fp64 path)
@@ -363,9 +363,11 @@ __device__ __forceinline__ void aq_prefetch(const ActArgs& a, int u, int q) {
                      static_cast<uint32_t>(min(a.group_rows, a.M - r0)) * a.K * 2);
 }
 
-// WIDE: the team is one or more whole warps (K >= 1024).
-template <int GRP, bool NORM, bool WIDE>
-__global__ void __launch_bounds__(32 * AQ_MAX_CWARPS, 1)
+// WIDE: the team is one or more whole warps (K >= 1024).  NW: warps per CTA,
+// 24 (up to 80 registers per thread) or 32 (up to 64), chosen by the host for
+// teams whose width divides it.
+template <int GRP, bool NORM, bool WIDE, int NW>
+__global__ void __launch_bounds__(32 * NW, 1)
     actquant_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     ActArgs a) {
   static_assert(GRP == 0 || GRP == 16 || GRP == 256, "group size 0, 16 or 256");

@@ -298,9 +298,9 @@ convrot_status launch_rowquant_pre(RowQuantArgs& a, int group, cudaStream_t st) 
 // token rows each, teams of eight threads per 256-element group.  The rows
 // are staged as [rows][K / 64][64] boxes and the norm weight as [K / 32][32]
 // lines, both with the 128-byte swizzle.
-template <int GRP, bool NORM, bool WIDE>
+template <int GRP, bool NORM, bool WIDE, int NW>
 convrot_status launch_actquant_w(const ActArgs& a, const float* norm_w, cudaStream_t st) {
-  auto k = actquant_kernel<GRP, NORM, WIDE>;
+  auto k = actquant_kernel<GRP, NORM, WIDE, NW>;
   const DeviceInfo d = current_device();
   if (d.device < 0 || d.sms <= 0) return CONVROT_ERR_CUDA;
   CUtensorMap mx, mw;
@@ -332,11 +332,15 @@ convrot_status launch_actquant_w(const ActArgs& a, const float* norm_w, cudaStre
   return launch_pdl(k, dim3(grid), dim3(a.team * a.rows), dyn, st, 1, mx, mw, a);
 }
 
-// teams of whole warps (K >= 1024) reduce with redux and a fixed shuffle tree
+// teams of whole warps (K >= 1024) reduce with redux and a fixed shuffle
+// tree; a CTA of 32 warps (64 registers per thread) where the plan filled
+// more than 24 warps, otherwise 24 (80 registers)
 template <int GRP, bool NORM>
 convrot_status launch_actquant_t(const ActArgs& a, const float* norm_w, cudaStream_t st) {
-  return a.team >= 32 ? launch_actquant_w<GRP, NORM, true>(a, norm_w, st)
-                      : launch_actquant_w<GRP, NORM, false>(a, norm_w, st);
+  const bool w32 = a.team * a.rows > 32 * 24;
+  if (a.team < 32) return launch_actquant_w<GRP, NORM, false, 24>(a, norm_w, st);
+  return w32 ? launch_actquant_w<GRP, NORM, true, 32>(a, norm_w, st)
+             : launch_actquant_w<GRP, NORM, true, 24>(a, norm_w, st);
 }
 
 // Team and stage plan of the activation kernel: eight threads per (virtual)
@@ -358,7 +362,10 @@ bool plan_actquant(int M, int K, int group, bool norm, int sms, ActArgs& a) {
   }
   if (team > 32 * AQ_MAX_TEAM_WARPS) return false;
   const int team_warps = std::max(1, team / 32);
-  const int max_rows = team >= 32 ? AQ_MAX_CWARPS / team_warps : AQ_MAX_CWARPS * (32 / team);
+  // 32 warps per CTA (64 registers) for whole-warp teams whose width divides
+  // 32 warps; 24 warps (80 registers) otherwise
+  const int cta_warps = (team >= 32 && 32 % team_warps == 0) ? 32 : 24;
+  const int max_rows = team >= 32 ? cta_warps / team_warps : cta_warps * (32 / team);
   const int per_sm = (M + std::max(1, sms) - 1) / std::max(1, sms);
   int rows = std::max(1, std::min(max_rows, per_sm));
   if (team < 32) rows = (rows * team + 31) / 32 * 32 / team;  // whole consumer warps
