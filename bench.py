@@ -105,7 +105,7 @@ def load_peaks():
 # helpers and the ABI file that plans and launches it
 KERNEL_SOURCES = {
     "gemm": ("gemm.cuh", "gemm2sm.cuh", "ptx.cuh", "convrot_abi.cu"),
-    "rotate_quant_act": ("rowquant.cuh", "ptx.cuh", "convrot_abi.cu"),
+    "rotate_quant_act": ("actquant.cuh", "rowquant.cuh", "ptx.cuh", "convrot_abi.cu"),
 }
 
 

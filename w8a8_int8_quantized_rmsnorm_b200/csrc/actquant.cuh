@@ -12,7 +12,8 @@
 // swizzle: thread 0 fills the ring at the start, and afterwards the warp that
 // releases a slot last (a shared counter per slot) refills it with the unit
 // `stages` steps later and prefetches the one after into L2.  No warp is set
-// aside for the copies, so the CTA's 24 warps share the registers four ways.
+// aside for the copies: a CTA of 24 warps gets up to 80 registers per thread,
+// one of 32 warps (for teams whose width in warps divides 32) up to 64.
 // The fp32 norm weight is copied once per CTA the same way, as lines of 32
 // values.  The swizzle (16-byte chunk c of
 // 128-byte line r stored at chunk c ^ (r & 7)) puts the eight threads of a

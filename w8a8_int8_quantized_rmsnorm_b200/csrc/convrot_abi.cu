@@ -130,10 +130,10 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t row
 
 // An N-d tiled map (N <= 3) of elements of `esize` bytes with the given
 // dimensions (innermost first), byte strides of dimensions 1..N-1, box and
-// swizzle; cached per thread like make_map.
+// swizzle mode; cached per thread like make_map.
 bool make_map_nd(CUtensorMap* map, const void* base, int rank, CUtensorMapDataType dtype,
                  int esize, const uint64_t* dims, const uint64_t* strides, const uint32_t* box,
-                 bool swizzle128) {
+                 CUtensorMapSwizzle swizzle) {
   struct Key {
     const void* base;
     int rank, dtype, esize, swz;
@@ -157,7 +157,7 @@ bool make_map_nd(CUtensorMap* map, const void* base, int rank, CUtensorMapDataTy
   key.rank = rank;
   key.dtype = static_cast<int>(dtype);
   key.esize = esize;
-  key.swz = swizzle128 ? 1 : 0;
+  key.swz = static_cast<int>(swizzle);
   for (int i = 0; i < rank; ++i) {
     key.dims[i] = dims[i];
     key.box[i] = box[i];
@@ -179,8 +179,7 @@ bool make_map_nd(CUtensorMap* map, const void* base, int rank, CUtensorMapDataTy
     if (i + 1 < rank) st[i] = strides[i];
   }
   const CUresult r = fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st,
-                        bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
   Entry& e = cache[next];
@@ -307,13 +306,15 @@ convrot_status launch_actquant_w(const ActArgs& a, const float* norm_w, cudaStre
   const uint64_t xdims[3] = {64, static_cast<uint64_t>(a.K / 64), static_cast<uint64_t>(a.M)};
   const uint64_t xstr[2] = {128, static_cast<uint64_t>(a.K) * 2};
   const uint32_t xbox[3] = {64, static_cast<uint32_t>(a.K / 64), static_cast<uint32_t>(a.group_rows)};
-  if (!make_map_nd(&mx, a.x, 3, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xdims, xstr, xbox, true))
+  if (!make_map_nd(&mx, a.x, 3, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xdims, xstr, xbox,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return CONVROT_ERR_CUDA;
   if (NORM) {
     const uint64_t wdims[2] = {32, static_cast<uint64_t>(a.K / 32)};
     const uint64_t wstr[1] = {128};
     const uint32_t wbox[2] = {32, static_cast<uint32_t>(a.w_box_lines)};
-    if (!make_map_nd(&mw, norm_w, 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, wdims, wstr, wbox, true))
+    if (!make_map_nd(&mw, norm_w, 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, wdims, wstr, wbox,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
       return CONVROT_ERR_CUDA;
   } else {
     std::memset(&mw, 0, sizeof(mw));
@@ -610,7 +611,7 @@ size_t ws_bytes(const GemmPlan& p) {
 template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
 convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
                              GemmArgs a, int grid, cudaStream_t st) {
-  using SM = GemmSmem<BN, W4 || WBF, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0>;
+  using SM = GemmSmem<BN, W4 || WBF, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0, WBF && SWAP>;
   auto k = gemm_kernel<BN, SWAP, W4, EPI, WBF>;
   // as many stages as fit next to the epilogue staging and the barriers in
   // 227 KB; at least ~116 KB so that a second CTA never shares the SM's TMEM
@@ -658,12 +659,16 @@ convrot_status run_gemm_wbf(const void* Xr, const int8_t* Wq, const float* s_row
   CUtensorMap mx, mw, my;
   std::memset(&my, 0, sizeof(my));
   // K atoms of 64 elements: 128 bytes of a bf16 row (swizzled like the int8
-  // atoms), 64 bytes of an int8 weight row (expanded in shared memory)
+  // atoms), 64 bytes of an int8 weight row (expanded in shared memory);
+  // swapped roles: the stage's two weight atoms land as one box of 128 rows x
+  // 128 bytes with the 128-byte swizzle and are expanded into tensor memory
   const uint32_t x_box_rows = p.swap ? bn : GEMM_BM;
   const uint32_t w_box_rows = p.swap ? GEMM_BM : bn;
   if (!make_map(&mx, Xr, M, K, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_box_rows, GEMM_BK / 2, true))
     return CONVROT_ERR_CUDA;
-  if (!make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK / 2, false)) return CONVROT_ERR_CUDA;
+  const bool wok = p.swap ? make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK, true)
+                          : make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK / 2, false);
+  if (!wok) return CONVROT_ERR_CUDA;
   bool ok;
   if (!p.swap) {
     ok = f32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32, true)

@@ -62,9 +62,10 @@ __host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
   return w4 ? (pair ? 2 : 1) : ((pair || swap) ? 2 : 1);
 }
 
-// K atoms per stage of the weight-only path: two for the small token tiles of
-// the swapped roles (a stage then stays near 52 KB), one otherwise.
-__host__ __device__ constexpr int wbf_katoms(bool swap, int bn) { return (swap && bn <= 64) ? 2 : 1; }
+// K atoms per stage of the weight-only path: two for the swapped roles (whose
+// expanded weights live in tensor memory, so a stage holds only the landed
+// int8 weights and the tokens), one otherwise.
+__host__ __device__ constexpr int wbf_katoms(bool swap, int) { return swap ? 2 : 1; }
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
 // SiLU(gate) * up of the MLP boundary: the weight rows alternate in blocks of
@@ -188,24 +189,37 @@ __device__ __forceinline__ void swiglu16(const uint32_t (&r)[32], float st, cons
 // per stage.  A converter stage's packed weight atom (64 bytes per row) lands
 // in the upper half of its weight atom's slot and is expanded in place to the
 // 128-byte swizzled rows the MMA reads, so a stage holds no separate packed
-// area.
-template <int BN, bool W4, bool SWAP, int KAO = 0>
+// area.  TSA (weight-only path, swapped roles): the stage's weights are only
+// the landed int8 tile (two 64-element atoms = 128 bytes per row, 128-byte
+// swizzle); their bf16 expansion is the MMA's A operand in tensor memory,
+// TSA_BUFS stages' worth of columns after the two accumulator buffers.
+template <int BN, bool W4, bool SWAP, int KAO = 0, bool TSA = false>
 struct GemmSmem {
   static constexpr int KA = KAO ? KAO : gemm_katoms(W4, false, SWAP);
-  static constexpr int A_ATOM = GEMM_BM * GEMM_BK;  // one 128-byte K atom of the A tile
+  // one K atom of the A tile: 128 bytes per row, or the landed 64 of TSA
+  static constexpr int A_ATOM = TSA ? GEMM_BM * (GEMM_BK / 2) : GEMM_BM * GEMM_BK;
   static constexpr int B_ATOM = BN * GEMM_BK;
   static constexpr int A_BYTES = KA * A_ATOM;
   static constexpr int B_BYTES = KA * B_ATOM;
   static constexpr int W_ROWS = SWAP ? GEMM_BM : BN;                // rows of the weight tile
   static constexpr int P_ATOM = W4 ? W_ROWS * (GEMM_BK / 2) : 0;  // packed int4 / int8 weight atom
   static constexpr int P_BYTES = KA * P_ATOM;                      // packed bytes per stage
-  static constexpr int PACKED_OFF = W_ROWS * (GEMM_BK / 2);        // inside a weight atom's slot
+  static constexpr int PACKED_OFF = TSA ? 0 : W_ROWS * (GEMM_BK / 2);  // inside a weight atom's slot
   static constexpr int STAGE = A_BYTES + B_BYTES;
   // per epilogue warp two 4 KB staging buffers (32 rows x 128 B) for output
   // stores and split-tile reductions
   static constexpr int STAGING = 4 * 2 * 4096;
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;  // TMEM columns per accumulator buffer
-  static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
+  // TSA: A buffers of one stage each (64 bf16 = 32 columns per K atom), at
+  // most TSA_BUFS of them and fewer than the stages (the converter reuses a
+  // buffer once its stage's slot has been released, which must not have
+  // happened twice since)
+  static constexpr int TSA_BUFS = 4;
+  static constexpr int TSA_COLS = KA * (GEMM_BK / 4);
+  static constexpr int TSA_COL0 = 2 * ACC_STRIDE;
+  static constexpr int TMEM_COLS = TSA ? 512 : 2 * ACC_STRIDE;
+  static_assert(!TSA || TSA_COL0 + TSA_BUFS * TSA_COLS <= 512, "tensor memory holds 512 columns");
+  static_assert(!TSA || KA == 2, "a TSA stage lands 128-byte weight rows: two bf16 atoms");
   static constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
   __host__ __device__ static int staging_offset(int stages) { return stages * STAGE; }
   __host__ __device__ static int bar_offset(int stages) { return stages * STAGE + STAGING; }
@@ -215,6 +229,25 @@ struct GemmSmem {
     return bar_offset(stages) + (3 * GEMM_MAX_STAGES + 7) * 8 + 64;
   }
 };
+
+// Four int8 codes q (one 32-bit word, lowest byte first) -> four bf16,
+// exactly, on the full-rate ALU: u = q + 128 (the sign bit flipped) goes into
+// the low byte of the fp32 2^23 + u, and subtracting 2^23 + 128 leaves q; q
+// has at most 8 significant bits, so its bf16 is the upper half.  lo holds
+// codes 0, 1 and hi codes 2, 3, the lower code in the low half of each.
+__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint64_t m01 = static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7540)) |
+                       (static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7541)) << 32);
+  const uint64_t m23 = static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7542)) |
+                       (static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7543)) << 32);
+  const uint64_t bias = 0x4B0000804B000080ull;  // (2^23 + 128, 2^23 + 128)
+  uint64_t f01, f23;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f01) : "l"(m01), "l"(bias));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f23) : "l"(m23), "l"(bias));
+  lo = __byte_perm(static_cast<uint32_t>(f01), static_cast<uint32_t>(f01 >> 32), 0x7632);
+  hi = __byte_perm(static_cast<uint32_t>(f23), static_cast<uint32_t>(f23 >> 32), 0x7632);
+}
 
 // Accumulator value: int32 for the integer MMAs, fp32 bits for kind::f16.
 template <bool F32ACC>
@@ -227,10 +260,13 @@ __device__ __forceinline__ float acc_value(uint32_t r) {
 // 255 (168) registers per thread is the most a launch can use.
 //
 // WBF (weight-only path): the activation operand is bf16 (already rotated),
-// the int8 weight tile is expanded to bf16 in shared memory by the converter
-// warps (the int4 path's staging: 64 bytes per row in, 128 bytes out, one
-// K atom = 64 elements per stage), the MMA is kind::f16 with an fp32
-// accumulator and the epilogue scales by s_row only.
+// the MMA is kind::f16 with an fp32 accumulator and the epilogue scales by
+// s_row only.  The int8 weight tile is expanded to bf16 by the converter
+// warps: for M > 128 in shared memory (the int4 path's staging: 64 bytes per
+// row in, 128 bytes out, one K atom = 64 elements per stage); for the swapped
+// roles into tensor memory as the MMA's A operand (TSA), each converter
+// thread taking one weight row of its warp's lane quadrant, so a stage's slot
+// holds only the landed int8 weights and the tokens.
 template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
 __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WBF) ? 168 : 255)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -238,7 +274,8 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
   constexpr bool CONV = W4 || WBF;  // a converter stage between TMA and the MMA
   static_assert(!(W4 && WBF), "int4 weights have no weight-only path");
   static_assert(!(WBF && EPI == EPI_SWIGLU), "the weight-only path has no SwiGLU epilogue");
-  using SM = GemmSmem<BN, CONV, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0>;
+  constexpr bool TSA = WBF && SWAP;  // expanded weights in tensor memory
+  using SM = GemmSmem<BN, CONV, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0, TSA>;
   static_assert(!W4 || SM::KA == 1, "int4 stages hold one K atom");
   constexpr int CW = SM::CW;
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
@@ -248,6 +285,8 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int S = a.stages;
+  // TSA: tensor-memory A buffers in use, fewer than the stages
+  const int nbufs = TSA ? min(SM::TSA_BUFS, S - 1) : 1;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::bar_offset(S));
   uint64_t* empty = full + GEMM_MAX_STAGES;
   uint64_t* conv = empty + GEMM_MAX_STAGES;
@@ -305,11 +344,16 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
       int ta, tb;
       tile_coords(a, s0.tile, ta, tb);
       const int kend = min(s0.kb1, s0.kb0 + S + GEMM_PREFETCH_ATOMS / SM::KA);
-      for (int kb = s0.kb0; kb < kend; ++kb)
+      for (int kb = s0.kb0; kb < kend; ++kb) {
+        if (TSA) {  // one 128-byte box per weight row and stage
+          tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
+          continue;
+        }
         for (int j = 0; j < SM::KA; ++j) {
           const int atom = kb * SM::KA + j;
           tma_prefetch_l2_2d(&tmA, (W4 || WBF) ? atom * (GEMM_BK / 2) : atom * GEMM_BK, ta * GEMM_BM);
         }
+      }
     }
   }
   pdl_wait();  // operands, scales and the output may belong to the previous kernel
@@ -340,9 +384,10 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
       auto xa = [](int atom) { return (W4 && SWAP) || WBF ? atom * (GEMM_BK / 2) : atom * GEMM_BK; };
       auto xb = [](int atom) { return (W4 && !SWAP) || WBF ? atom * (GEMM_BK / 2) : atom * GEMM_BK; };
       auto prefetch = [&](int ta, int tb, int kb) {
+        if (TSA) tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
 #pragma unroll
         for (int j = 0; j < KA; ++j) {
-          tma_prefetch_l2_2d(&tmA, xa(kb * KA + j), ta * GEMM_BM);
+          if (!TSA) tma_prefetch_l2_2d(&tmA, xa(kb * KA + j), ta * GEMM_BM);
           tma_prefetch_l2_2d(&tmB, xb(kb * KA + j), tb * BN);
         }
       };
@@ -360,13 +405,17 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           }
           uint8_t* st = smem + s * SM::STAGE;
           mbar_arrive_expect_tx(&full[s], tx);
+          // TSA: the stage's weights as one box of 128 rows x 128 bytes (both
+          // 64-element atoms of each row)
+          if (TSA) tma_load_2d(st, &tmA, &full[s], kb * GEMM_BK, ta * GEMM_BM, pol_a);
 #pragma unroll
           for (int j = 0; j < KA; ++j) {
             // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
             const int atom = kb * KA + j;
             // a packed weight atom lands in the upper half of its slot
-            tma_load_2d(st + j * SM::A_ATOM + ((CONV && SWAP) ? SM::PACKED_OFF : 0), &tmA, &full[s],
-                        xa(atom), ta * GEMM_BM, pol_a);
+            if (!TSA)
+              tma_load_2d(st + j * SM::A_ATOM + ((CONV && SWAP) ? SM::PACKED_OFF : 0), &tmA,
+                          &full[s], xa(atom), ta * GEMM_BM, pol_a);
             tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM + ((CONV && !SWAP) ? SM::PACKED_OFF : 0),
                         &tmB, &full[s], xb(atom), tb * BN, pol_b);
           }
@@ -405,17 +454,23 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           tc_fence_after();
           const uint32_t sa = smem_addr(smem + s * SM::STAGE);
           const uint32_t sb = sa + SM::A_BYTES;
+          // TSA: this stage's expanded weights, 32 columns per K atom
+          const uint32_t ta = tmem_base + SM::TSA_COL0 + (it % nbufs) * SM::TSA_COLS;
 #pragma unroll
           for (int j = 0; j < SM::KA; ++j) {
 #pragma unroll
             for (int k = 0; k < GEMM_BK / GEMM_UMMA_K; ++k) {
-              const uint64_t ad = sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K);
               const uint64_t bd = sw128_kmajor_desc(sb + j * SM::B_ATOM + k * GEMM_UMMA_K);
               const uint32_t acc = (kb > seg.kb0 || j > 0 || k > 0) ? 1u : 0u;
-              if (WBF)
-                mma_bf16(d, ad, bd, IDESC, acc);
-              else
-                mma_s8(d, ad, bd, IDESC, acc);
+              if (TSA) {
+                mma_bf16_ts(d, ta + j * (GEMM_BK / 4) + k * (GEMM_UMMA_K / 4), bd, IDESC, acc);
+              } else {
+                const uint64_t ad = sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K);
+                if (WBF)
+                  mma_bf16(d, ad, bd, IDESC, acc);
+                else
+                  mma_s8(d, ad, bd, IDESC, acc);
+              }
             }
           }
           mma_commit(&empty[s]);
@@ -768,6 +823,61 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
     // the staged outputs must have been read before the CTA exits; the global
     // writes themselves complete before the grid does
     if (lane == 0) bulk_wait_group_read<0>();
+  } else if (TSA) {
+    // ------------------------------------------------------------ int8 -> bf16
+    // into tensor memory.  Warp w may access TMEM lanes 32 (w & 3) .. + 31:
+    // lane l of it expands weight row 32 (w & 3) + l of the tile.  The stage's
+    // rows landed as 128 bytes (atom j in chunks 4j .. 4j + 3) with the
+    // 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)), so each
+    // quarter-warp's 16-byte loads fall in eight different bank groups.
+    const int q = warp & 3;
+    const int r = 32 * q + lane;
+    const uint32_t tlane = static_cast<uint32_t>(32 * q) << 16;
+    const int rsw = r & 7;
+    uint32_t it = 0;
+    bool ok = true;
+    while (ok && sched.next(seg)) {
+      for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, SITE_CONV_FULL)) {
+          ok = false;
+          break;
+        }
+        const int x = static_cast<int>(it % static_cast<uint32_t>(nbufs));
+        if (it >= static_cast<uint32_t>(nbufs)) {
+          // buffer x last held stage it - nbufs: its MMAs are complete once that
+          // stage's slot was released (the release after it needs this stage's
+          // MMAs, so the parity is unambiguous)
+          const uint32_t prev = it - static_cast<uint32_t>(nbufs);
+          if (!mbar_wait(&empty[prev % S], (prev / S) & 1u, abort_flag, SITE_CONV_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const uint8_t* st = smem + s * SM::STAGE;
+        const uint32_t ta = tmem_base + tlane + SM::TSA_COL0 + x * SM::TSA_COLS;
+#pragma unroll
+        for (int j = 0; j < SM::KA; ++j) {
+          const uint8_t* row = st + r * GEMM_BK;
+          uint32_t o[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 pk = ld_shared_v4(row + (((4 * j + c) ^ rsw) << 4));
+            i8x4_to_bf16x4(pk.x, o[8 * c], o[8 * c + 1]);
+            i8x4_to_bf16x4(pk.y, o[8 * c + 2], o[8 * c + 3]);
+            i8x4_to_bf16x4(pk.z, o[8 * c + 4], o[8 * c + 5]);
+            i8x4_to_bf16x4(pk.w, o[8 * c + 6], o[8 * c + 7]);
+          }
+          tmem_st_32x32b_x32(ta + j * (GEMM_BK / 4), o);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&conv[s]);
+      }
+    }
   } else if (CONV) {
     // ------------------------------------------------------------ int4 unpack /
     // int8 -> bf16 (WBF).  Each thread reads its share of every packed atom of
@@ -823,21 +933,7 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             if (WBF) {
-              // four int8 codes q -> four bf16, exactly, on the full-rate ALU:
-              // u = q + 128 (the sign bit flipped) goes into the low byte of
-              // the fp32 2^23 + u, and subtracting 2^23 + 128 leaves q; q has
-              // at most 8 significant bits, so its bf16 is the upper half
-              const uint32_t u = w[h] ^ 0x80808080u;
-              const uint64_t m01 = static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7540)) |
-                                   (static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7541)) << 32);
-              const uint64_t m23 = static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7542)) |
-                                   (static_cast<uint64_t>(__byte_perm(u, 0x4B000000u, 0x7543)) << 32);
-              const uint64_t bias = 0x4B0000804B000080ull;  // (2^23 + 128, 2^23 + 128)
-              uint64_t f01, f23;
-              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f01) : "l"(m01), "l"(bias));
-              asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f23) : "l"(m23), "l"(bias));
-              o[2 * h] = __byte_perm(static_cast<uint32_t>(f01), static_cast<uint32_t>(f01 >> 32), 0x7632);
-              o[2 * h + 1] = __byte_perm(static_cast<uint32_t>(f23), static_cast<uint32_t>(f23 >> 32), 0x7632);
+              i8x4_to_bf16x4(w[h], o[2 * h], o[2 * h + 1]);
             } else {
               const uint32_t lo = (w[h] << 4) & 0xF0F0F0F0u;
               const uint32_t hi = w[h] & 0xF0F0F0F0u;
