@@ -49,7 +49,9 @@ constexpr int GEMM_BK = 128;  // int8 elements (bytes) of K per swizzle atom
 constexpr int GEMM_UMMA_K = 32;
 constexpr int GEMM_MAX_STAGES = 16;
 constexpr int GEMM_GROUP_A = 8;
-constexpr int GEMM_PREFETCH_ATOMS = 8;  // L2 prefetch this many K atoms beyond the ring
+// decode kernels: before the dependency wait, the weights of this many K atoms
+// beyond the ring's first fill go towards L2
+constexpr int GEMM_PREFETCH_ATOMS = 8;
 // 128-byte K atoms per pipeline stage.  A single thread issues every
 // tcgen05.mma, and each MMA issue, stage wait and commit costs that thread tens
 // of cycles: with one atom (four 32-deep MMAs) per stage the issuing thread
@@ -347,11 +349,12 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
       for (int kb = s0.kb0; kb < kend; ++kb) {
         if (TSA) {  // one 128-byte box per weight row and stage
           tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
-          continue;
-        }
-        for (int j = 0; j < SM::KA; ++j) {
-          const int atom = kb * SM::KA + j;
-          tma_prefetch_l2_2d(&tmA, (W4 || WBF) ? atom * (GEMM_BK / 2) : atom * GEMM_BK, ta * GEMM_BM);
+        } else {
+          for (int j = 0; j < SM::KA; ++j) {
+            const int atom = kb * SM::KA + j;
+            tma_prefetch_l2_2d(&tmA, (W4 || WBF) ? atom * (GEMM_BK / 2) : atom * GEMM_BK,
+                               ta * GEMM_BM);
+          }
         }
       }
     }
@@ -375,27 +378,17 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
       }
       uint32_t it = 0;
       bool ok = true;
-      // L2 prefetch distance in K steps: beyond what the shared ring holds, so
-      // that tiles first touched in DRAM are in L2 when their load is issued
       constexpr int KA = SM::KA;
-      const int pfd = S + GEMM_PREFETCH_ATOMS / KA;
       // innermost TMA coordinate of K atom `atom`: int8 bytes, or half of that
       // for packed int4 weights; WBF atoms are 64 elements of either operand
       auto xa = [](int atom) { return (W4 && SWAP) || WBF ? atom * (GEMM_BK / 2) : atom * GEMM_BK; };
       auto xb = [](int atom) { return (W4 && !SWAP) || WBF ? atom * (GEMM_BK / 2) : atom * GEMM_BK; };
-      auto prefetch = [&](int ta, int tb, int kb) {
-        if (TSA) tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
-#pragma unroll
-        for (int j = 0; j < KA; ++j) {
-          if (!TSA) tma_prefetch_l2_2d(&tmA, xa(kb * KA + j), ta * GEMM_BM);
-          tma_prefetch_l2_2d(&tmB, xb(kb * KA + j), tb * BN);
-        }
-      };
+      // No L2 prefetches run ahead of the ring: each prefetch request takes
+      // the same copy engine as the loads, and without them the decode GEMMs
+      // ran 8-9 % faster (measured at M = 1, 16 and 128).
       while (ok && sched.next(seg)) {
         int ta, tb;
         tile_coords(a, seg.tile, ta, tb);
-        // the first ring-full of loads goes out before the initial prefetch window
-        const int win = min(seg.kb1, seg.kb0 + S) - 1;
         for (int kb = seg.kb0; kb < seg.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1u;
@@ -419,9 +412,6 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
             tma_load_2d(st + SM::A_BYTES + j * SM::B_ATOM + ((CONV && !SWAP) ? SM::PACKED_OFF : 0),
                         &tmB, &full[s], xb(atom), tb * BN, pol_b);
           }
-          if (kb + pfd < seg.kb1) prefetch(ta, tb, kb + pfd);
-          if (kb == win)
-            for (int kp = seg.kb0 + S; kp < min(seg.kb1, seg.kb0 + pfd); ++kp) prefetch(ta, tb, kp);
         }
       }
       // drain: make sure no copy is still landing in shared memory when the CTA exits
