@@ -57,10 +57,11 @@ def test_rotate_act_bf16(cr, M, K, group, norm):
     assert np.all(err <= _tol.bf16_ulp(v) * 1.0001 + 2 * e32), f"worst {np.max(err - _tol.bf16_ulp(v)):.3e}"
 
 
-# (16, 20480, 1024) and (100, 20480, 4096) split the K range of some tiles over
+# (16, 20480, 4096) and (100, 20480, 4096) split the K range of some tiles over
 # two CTAs (stream-K with fp32 partial sums); the others run whole tiles
 SHAPES = [(1, 256, 256), (16, 1024, 4096), (40, 520, 1040), (128, 4096, 4096), (129, 264, 512),
-          (512, 4096, 4096), (1000, 1032, 2080), (16, 20480, 1024), (100, 20480, 4096)]
+          (512, 4096, 4096), (1000, 1032, 2080), (16, 20480, 1024), (16, 20480, 4096),
+          (100, 20480, 4096)]
 
 
 def _operands(M, N, K):
@@ -148,7 +149,7 @@ def test_weight_only_edge_cases(cr):
     assert not Y2[:, 5].any()
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 20480, 1024), (100, 20480, 4096)])
+@pytest.mark.parametrize("M,N,K", [(16, 20480, 4096), (100, 20480, 4096)])
 def test_weight_only_split_tiles_deterministic(cr, M, N, K):
     """Split tiles have at most two fp32 parts, so repeated calls agree bit for
     bit whatever the order the parts arrive in; the workspace is zero again."""

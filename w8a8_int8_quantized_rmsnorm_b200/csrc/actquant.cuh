@@ -11,12 +11,12 @@
 // stage of a [R rows][K / 64 lines][64 elements] box with the 128-byte
 // swizzle: thread 0 fills the ring at the start, and afterwards the warp that
 // releases a slot last (a shared counter per slot) refills it with the unit
-// `stages` steps later and prefetches the one after into L2.  No warp is set
-// aside for the copies: a CTA of 24 warps gets up to 80 registers per thread,
-// one of 32 warps (for teams whose width in warps divides 32) up to 64.
-// The fp32 norm weight is copied once per CTA the same way, as lines of 32
-// values.  The swizzle (16-byte chunk c of
-// 128-byte line r stored at chunk c ^ (r & 7)) puts the eight threads of a
+// `stages` steps later (and, with the norm, prefetches the one after into
+// L2).  No warp is set aside for the copies: a CTA of 24 warps gets up to 80
+// registers per thread, one of 32 warps (for teams whose width in warps
+// divides 32) up to 64.  The fp32 norm weight is copied once per CTA the same
+// way, as lines of 32 values.  The swizzle (16-byte chunk c of 128-byte line
+// r stored at chunk c ^ (r & 7)) puts the eight threads of a
 // group, which read 64 bytes of the row (and 128 bytes of the weight) each,
 // in eight different bank groups.
 // The consumer warps form R teams, one row each; a row's 256-element groups
@@ -372,6 +372,11 @@ __global__ void __launch_bounds__(32 * NW, 1)
     actquant_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                     ActArgs a) {
   static_assert(GRP == 0 || GRP == 16 || GRP == 256, "group size 0, 16 or 256");
+  // L2 prefetch of the unit after the ring's next one.  Without the norm it
+  // only takes the copy engine from the ring's own copies (measured without
+  // it: 8192 x 4096 24.0 -> 23.0 us); with the norm, dropping it costs the
+  // 32-warp build registers (more spills) and 4 % at 2048 x 4096, so it stays.
+  constexpr bool AQ_L2_PREFETCH = NORM;
   // K is a multiple of 256 with 256-point groups: no per-element bounds checks
   constexpr bool WHOLE = GRP == 256;
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
@@ -428,7 +433,7 @@ __global__ void __launch_bounds__(32 * NW, 1)
                  &issued[q * a.stages + j], u, q);
     }
     const int uf = blockIdx.x + a.stages * gridDim.x;
-    if (uf < units)
+    if (AQ_L2_PREFETCH && uf < units)
       for (int q = 0; q < ngroups; ++q) aq_prefetch(a, uf, q);
   }
   // ------------------------------------------------------------ consumers
@@ -459,7 +464,7 @@ __global__ void __launch_bounds__(32 * NW, 1)
   unsigned* qrel = released + q * a.stages;
   unsigned* qiss = issued + q * a.stages;
   // the warp of the group that releases a ring slot last refills it with the
-  // group's rows `stages` units later and warms L2 with the unit after that
+  // group's rows `stages` units later (and may warm L2 with the unit after that)
   auto release = [&](int s, int u) {
     __syncwarp();
     if (lane == 0) {
@@ -470,7 +475,7 @@ __global__ void __launch_bounds__(32 * NW, 1)
         const int un = u + a.stages * static_cast<int>(gridDim.x);
         if (un < units) aq_issue(&tmX, a, ring + s * a.slot_stride, &qfull[s], &qiss[s], un, q);
         const int uf = un + static_cast<int>(gridDim.x);
-        if (uf < units) aq_prefetch(a, uf, q);
+        if (AQ_L2_PREFETCH && uf < units) aq_prefetch(a, uf, q);
       }
     }
   };

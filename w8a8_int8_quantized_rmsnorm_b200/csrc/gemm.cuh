@@ -64,10 +64,15 @@ __host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
   return w4 ? (pair ? 2 : 1) : ((pair || swap) ? 2 : 1);
 }
 
-// K atoms per stage of the weight-only path: two for the swapped roles (whose
-// expanded weights live in tensor memory, so a stage holds only the landed
-// int8 weights and the tokens), one otherwise.
-__host__ __device__ constexpr int wbf_katoms(bool swap, int) { return swap ? 2 : 1; }
+// K atoms per stage of the weight-only path.  The swapped roles expand their
+// weights into tensor memory, so a stage holds only the landed int8 weights
+// and the tokens: four atoms (32 KB of weights, the int8 decode stage's
+// share) for token tiles up to 64, two for 128 (where four would leave two
+// stages).  Halving the stages per weight byte took M = 16 from 37.6 to
+// 30.7 us (measured).  One atom otherwise.
+__host__ __device__ constexpr int wbf_katoms(bool swap, int bn) {
+  return swap ? (bn <= 64 ? 4 : 2) : 1;
+}
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
 // SiLU(gate) * up of the MLP boundary: the weight rows alternate in blocks of
@@ -192,9 +197,10 @@ __device__ __forceinline__ void swiglu16(const uint32_t (&r)[32], float st, cons
 // in the upper half of its weight atom's slot and is expanded in place to the
 // 128-byte swizzled rows the MMA reads, so a stage holds no separate packed
 // area.  TSA (weight-only path, swapped roles): the stage's weights are only
-// the landed int8 tile (two 64-element atoms = 128 bytes per row, 128-byte
-// swizzle); their bf16 expansion is the MMA's A operand in tensor memory,
-// TSA_BUFS stages' worth of columns after the two accumulator buffers.
+// the landed int8 tile (boxes of two 64-element atoms = 128 bytes per row,
+// 128-byte swizzle); their bf16 expansion is the MMA's A operand in tensor
+// memory, up to TSA_BUFS stages' worth of columns after the two accumulator
+// buffers.
 template <int BN, bool W4, bool SWAP, int KAO = 0, bool TSA = false>
 struct GemmSmem {
   static constexpr int KA = KAO ? KAO : gemm_katoms(W4, false, SWAP);
@@ -220,8 +226,9 @@ struct GemmSmem {
   static constexpr int TSA_COLS = KA * (GEMM_BK / 4);
   static constexpr int TSA_COL0 = 2 * ACC_STRIDE;
   static constexpr int TMEM_COLS = TSA ? 512 : 2 * ACC_STRIDE;
-  static_assert(!TSA || TSA_COL0 + TSA_BUFS * TSA_COLS <= 512, "tensor memory holds 512 columns");
-  static_assert(!TSA || KA == 2, "a TSA stage lands 128-byte weight rows: two bf16 atoms");
+  static constexpr int TSA_MAXBUF = (512 - TSA_COL0) / TSA_COLS;  // what tensor memory holds
+  static_assert(!TSA || TSA_MAXBUF >= 1, "tensor memory holds 512 columns");
+  static_assert(!TSA || KA % 2 == 0, "a TSA stage lands 128-byte weight rows: two bf16 atoms");
   static constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
   __host__ __device__ static int staging_offset(int stages) { return stages * STAGE; }
   __host__ __device__ static int bar_offset(int stages) { return stages * STAGE + STAGING; }
@@ -288,7 +295,7 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
                                              ~static_cast<uintptr_t>(1023));
   const int S = a.stages;
   // TSA: tensor-memory A buffers in use, fewer than the stages
-  const int nbufs = TSA ? min(SM::TSA_BUFS, S - 1) : 1;
+  const int nbufs = TSA ? min(min(SM::TSA_BUFS, S - 1), SM::TSA_MAXBUF) : 1;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::bar_offset(S));
   uint64_t* empty = full + GEMM_MAX_STAGES;
   uint64_t* conv = empty + GEMM_MAX_STAGES;
@@ -347,8 +354,9 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
       tile_coords(a, s0.tile, ta, tb);
       const int kend = min(s0.kb1, s0.kb0 + S + GEMM_PREFETCH_ATOMS / SM::KA);
       for (int kb = s0.kb0; kb < kend; ++kb) {
-        if (TSA) {  // one 128-byte box per weight row and stage
-          tma_prefetch_l2_2d(&tmA, kb * GEMM_BK, ta * GEMM_BM);
+        if (TSA) {  // 128-byte boxes per weight row
+          for (int h = 0; h < SM::KA / 2; ++h)
+            tma_prefetch_l2_2d(&tmA, (kb * SM::KA / 2 + h) * GEMM_BK, ta * GEMM_BM);
         } else {
           for (int j = 0; j < SM::KA; ++j) {
             const int atom = kb * SM::KA + j;
@@ -398,9 +406,12 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           }
           uint8_t* st = smem + s * SM::STAGE;
           mbar_arrive_expect_tx(&full[s], tx);
-          // TSA: the stage's weights as one box of 128 rows x 128 bytes (both
-          // 64-element atoms of each row)
-          if (TSA) tma_load_2d(st, &tmA, &full[s], kb * GEMM_BK, ta * GEMM_BM, pol_a);
+          // TSA: the stage's weights as boxes of 128 rows x 128 bytes (two
+          // 64-element atoms of each row per box)
+          if (TSA)
+            for (int h = 0; h < KA / 2; ++h)
+              tma_load_2d(st + h * (GEMM_BM * GEMM_BK), &tmA, &full[s], (kb * KA / 2 + h) * GEMM_BK,
+                          ta * GEMM_BM, pol_a);
 #pragma unroll
           for (int j = 0; j < KA; ++j) {
             // atoms past K read as zeros (TMA out-of-bounds fill) and add nothing
@@ -817,9 +828,10 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
     // ------------------------------------------------------------ int8 -> bf16
     // into tensor memory.  Warp w may access TMEM lanes 32 (w & 3) .. + 31:
     // lane l of it expands weight row 32 (w & 3) + l of the tile.  The stage's
-    // rows landed as 128 bytes (atom j in chunks 4j .. 4j + 3) with the
-    // 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)), so each
-    // quarter-warp's 16-byte loads fall in eight different bank groups.
+    // rows landed in boxes of 128 bytes per row (atom j in box j / 2, chunks
+    // 4 (j & 1) .. + 3) with the 128-byte swizzle (16-byte chunk c of row r at
+    // chunk c ^ (r & 7)), so each quarter-warp's 16-byte loads fall in eight
+    // different bank groups.
     const int q = warp & 3;
     const int r = 32 * q + lane;
     const uint32_t tlane = static_cast<uint32_t>(32 * q) << 16;
@@ -850,11 +862,11 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
         const uint32_t ta = tmem_base + tlane + SM::TSA_COL0 + x * SM::TSA_COLS;
 #pragma unroll
         for (int j = 0; j < SM::KA; ++j) {
-          const uint8_t* row = st + r * GEMM_BK;
+          const uint8_t* row = st + (j >> 1) * (GEMM_BM * GEMM_BK) + r * GEMM_BK;
           uint32_t o[32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const uint4 pk = ld_shared_v4(row + (((4 * j + c) ^ rsw) << 4));
+            const uint4 pk = ld_shared_v4(row + (((4 * (j & 1) + c) ^ rsw) << 4));
             i8x4_to_bf16x4(pk.x, o[8 * c], o[8 * c + 1]);
             i8x4_to_bf16x4(pk.y, o[8 * c + 2], o[8 * c + 3]);
             i8x4_to_bf16x4(pk.z, o[8 * c + 4], o[8 * c + 5]);
