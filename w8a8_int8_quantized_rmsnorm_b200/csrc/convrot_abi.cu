@@ -430,15 +430,16 @@ int pick_bn_swap(int M) {
 // kernel, CTA pairs (clusters of two) for the pair kernel.
 // `clusters4` is the number of co-resident four-CTA clusters of the split
 // pair kernel (0 if unavailable).
-// wbf: the weight-only path (bf16 activations, int8 weights expanded to bf16,
-// fp32 accumulators): single-CTA tiles, 64 K elements per stage; stream-K
-// only for the swapped roles and only where every split tile has at most two
-// parts (each unit's share is at least a whole tile), so that the fp32 sum of
-// the parts does not depend on their order.
+// wbf: the weight-only path (bf16 activations, int8 weights expanded to bf16
+// in tensor memory, fp32 accumulators): swapped roles at every M (weights as
+// the MMA's A operand, token tiles of up to 128 as B), K atoms of 64
+// elements; stream-K only where every split tile has at most two parts (each
+// unit's share is at least a whole tile), so that the fp32 sum of the parts
+// does not depend on their order.
 GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int clusters4,
                    bool wbf = false) {
   GemmPlan p{};
-  p.swap = M <= 128;
+  p.swap = M <= 128 || wbf;
   p.pair = !p.swap && pairs > 0 && !wbf;
   p.bn = p.swap ? pick_bn_swap(M) : 256;
   const int rowsA = p.swap ? N : M;
@@ -447,7 +448,7 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   p.tilesA = (rowsA + tileA - 1) / tileA;
   p.tilesB = (rowsB + p.bn - 1) / p.bn;
   p.num_tiles = p.tilesA * p.tilesB;
-  const int stage_k = wbf ? (GEMM_BK / 2) * wbf_katoms(p.swap, p.bn)
+  const int stage_k = wbf ? (GEMM_BK / 2) * wbf_katoms(p.bn)
                           : GEMM_BK * gemm_katoms(w4, p.pair, p.swap);
   p.num_kb = (K + stage_k - 1) / stage_k;
   // One wave of 256 x 256 tiles that fits the co-resident clusters: each tile
@@ -479,7 +480,7 @@ GemmPlan plan_gemm(int M, int N, int K, int sms, int pairs, bool w4, int cluster
   const long long t_sk = static_cast<long long>(p.dp_tiles / p.grid) * p.num_kb +
                          (sk_total + p.grid - 1) / p.grid + fixup_stages(p.swap, p.bn);
   const bool two_parts = sk_tiles * p.num_kb / p.grid >= p.num_kb;
-  if ((wbf && (!p.swap || !two_parts)) || t_dp <= t_sk) {
+  if ((wbf && !two_parts) || t_dp <= t_sk) {
     p.dp_tiles = p.num_tiles;
     sk_tiles = 0;
   }
@@ -611,7 +612,7 @@ size_t ws_bytes(const GemmPlan& p) {
 template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
 convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& my,
                              GemmArgs a, int grid, cudaStream_t st) {
-  using SM = GemmSmem<BN, W4 || WBF, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0, WBF && SWAP>;
+  using SM = GemmSmem<BN, W4 || WBF, SWAP, WBF ? wbf_katoms(BN) : 0, WBF>;
   auto k = gemm_kernel<BN, SWAP, W4, EPI, WBF>;
   // as many stages as fit next to the epilogue staging and the barriers in
   // 227 KB; at least ~116 KB so that a second CTA never shares the SM's TMEM
@@ -633,9 +634,8 @@ convrot_status launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const
 }
 
 template <int EPI>
-convrot_status launch_wbf(bool swap, int bn, const CUtensorMap& ma, const CUtensorMap& mb,
+convrot_status launch_wbf(int bn, const CUtensorMap& ma, const CUtensorMap& mb,
                           const CUtensorMap& my, const GemmArgs& a, int grid, cudaStream_t st) {
-  if (!swap) return launch_gemm_t<256, false, false, EPI, true>(ma, mb, my, a, grid, st);
   switch (bn) {
     case 16: return launch_gemm_t<16, true, false, EPI, true>(ma, mb, my, a, grid, st);
     case 32: return launch_gemm_t<32, true, false, EPI, true>(ma, mb, my, a, grid, st);
@@ -658,33 +658,24 @@ convrot_status run_gemm_wbf(const void* Xr, const int8_t* Wq, const float* s_row
   const int bn = p.bn;
   CUtensorMap mx, mw, my;
   std::memset(&my, 0, sizeof(my));
-  // K atoms of 64 elements: 128 bytes of a bf16 row (swizzled like the int8
-  // atoms), 64 bytes of an int8 weight row (expanded in shared memory);
-  // swapped roles: the stage's two weight atoms land as one box of 128 rows x
-  // 128 bytes with the 128-byte swizzle and are expanded into tensor memory
-  const uint32_t x_box_rows = p.swap ? bn : GEMM_BM;
-  const uint32_t w_box_rows = p.swap ? GEMM_BM : bn;
-  if (!make_map(&mx, Xr, M, K, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_box_rows, GEMM_BK / 2, true))
+  // swapped roles: token atoms of 64 elements (128 bytes of a bf16 row,
+  // swizzled like the int8 atoms); the weights land as boxes of 128 rows x
+  // 128 bytes (two atoms) with the 128-byte swizzle and are expanded into
+  // tensor memory
+  if (!make_map(&mx, Xr, M, K, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bn, GEMM_BK / 2, true))
     return CONVROT_ERR_CUDA;
-  const bool wok = p.swap ? make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK, true)
-                          : make_map_u8(&mw, Wq, N, K, w_box_rows, GEMM_BK / 2, false);
-  if (!wok) return CONVROT_ERR_CUDA;
-  bool ok;
-  if (!p.swap) {
-    ok = f32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 32, 32, true)
-                 : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, 64, true);
-  } else {
-    const uint32_t cw = bn < 32 ? bn : 32;
-    ok = f32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cw, 128, false)
-                 : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cw, 128, false);
-  }
+  if (!make_map_u8(&mw, Wq, N, K, GEMM_BM, GEMM_BK, true)) return CONVROT_ERR_CUDA;
+  // the output as chunks of up to 32 tokens x 128 columns, unswizzled
+  const uint32_t cw = bn < 32 ? bn : 32;
+  const bool ok = f32_out ? make_map(&my, out, M, N, 4, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cw, 128, false)
+                          : make_map(&my, out, M, N, 2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cw, 128, false);
   if (!ok) return CONVROT_ERR_CUDA;
   GemmArgs a{};
   a.M = M;
   a.N = N;
   a.K = K;
-  a.rowsA = p.swap ? N : M;
-  a.rowsB = p.swap ? M : N;
+  a.rowsA = N;
+  a.rowsB = M;
   a.tilesA = p.tilesA;
   a.tilesB = p.tilesB;
   a.num_tiles = p.num_tiles;
@@ -700,10 +691,8 @@ convrot_status run_gemm_wbf(const void* Xr, const int8_t* Wq, const float* s_row
   a.s_row = s_row;
   a.srow_vec = (s_row != nullptr && aligned(s_row, 16)) ? 1 : 0;
   a.out = out;
-  const CUtensorMap& ma = p.swap ? mw : mx;
-  const CUtensorMap& mb = p.swap ? mx : mw;
-  return f32_out ? launch_wbf<EPI_S32>(p.swap, bn, ma, mb, my, a, p.grid, st)
-                 : launch_wbf<EPI_BF16>(p.swap, bn, ma, mb, my, a, p.grid, st);
+  return f32_out ? launch_wbf<EPI_S32>(bn, mw, mx, my, a, p.grid, st)
+                 : launch_wbf<EPI_BF16>(bn, mw, mx, my, a, p.grid, st);
 }
 
 template <bool SWAP, bool W4, int EPI>

@@ -64,15 +64,13 @@ __host__ __device__ constexpr int gemm_katoms(bool w4, bool pair, bool swap) {
   return w4 ? (pair ? 2 : 1) : ((pair || swap) ? 2 : 1);
 }
 
-// K atoms per stage of the weight-only path.  The swapped roles expand their
-// weights into tensor memory, so a stage holds only the landed int8 weights
-// and the tokens: four atoms (32 KB of weights, the int8 decode stage's
-// share) for token tiles up to 64, two for 128 (where four would leave two
-// stages).  Halving the stages per weight byte took M = 16 from 37.6 to
-// 30.7 us (measured).  One atom otherwise.
-__host__ __device__ constexpr int wbf_katoms(bool swap, int bn) {
-  return swap ? (bn <= 64 ? 4 : 2) : 1;
-}
+// K atoms (64 elements each) per stage of the weight-only path.  Its weights
+// are expanded into tensor memory, so a stage holds only the landed int8
+// weights and the tokens: four atoms (32 KB of weights, the int8 decode
+// stage's share) for token tiles up to 64, two for 128 (where four would
+// leave two stages).  Halving the stages per weight byte took M = 16 from
+// 37.6 to 30.7 us (measured).
+__host__ __device__ constexpr int wbf_katoms(int bn) { return bn <= 64 ? 4 : 2; }
 constexpr int EPI_BF16 = 0;
 constexpr int EPI_S32 = 1;
 // SiLU(gate) * up of the MLP boundary: the weight rows alternate in blocks of
@@ -268,14 +266,14 @@ __device__ __forceinline__ float acc_value(uint32_t r) {
 // CTA's warps spread over four): with 6 (10) warps, two (three) share one, so
 // 255 (168) registers per thread is the most a launch can use.
 //
-// WBF (weight-only path): the activation operand is bf16 (already rotated),
-// the MMA is kind::f16 with an fp32 accumulator and the epilogue scales by
-// s_row only.  The int8 weight tile is expanded to bf16 by the converter
-// warps: for M > 128 in shared memory (the int4 path's staging: 64 bytes per
-// row in, 128 bytes out, one K atom = 64 elements per stage); for the swapped
-// roles into tensor memory as the MMA's A operand (TSA), each converter
-// thread taking one weight row of its warp's lane quadrant, so a stage's slot
-// holds only the landed int8 weights and the tokens.
+// WBF (weight-only path, always the swapped roles): the activation operand is
+// bf16 (already rotated), the MMA is kind::f16 with an fp32 accumulator and
+// the epilogue scales by s_row only.  The converter warps expand the int8
+// weight tile to bf16 into tensor memory as the MMA's A operand (TSA), each
+// converter thread taking one weight row of its warp's lane quadrant, so a
+// stage's slot holds only the landed int8 weights and the tokens.  (Expanding
+// into shared memory, as the int4 path does, measured 2x slower at M = 512,
+// N = K = 4096 and 5 % slower at M = 2048, N = 24576.)
 template <int BN, bool SWAP, bool W4, int EPI, bool WBF = false>
 __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WBF) ? 168 : 255)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -283,8 +281,9 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
   constexpr bool CONV = W4 || WBF;  // a converter stage between TMA and the MMA
   static_assert(!(W4 && WBF), "int4 weights have no weight-only path");
   static_assert(!(WBF && EPI == EPI_SWIGLU), "the weight-only path has no SwiGLU epilogue");
-  constexpr bool TSA = WBF && SWAP;  // expanded weights in tensor memory
-  using SM = GemmSmem<BN, CONV, SWAP, WBF ? wbf_katoms(SWAP, BN) : 0, TSA>;
+  static_assert(!WBF || SWAP, "the weight-only path runs the swapped roles");
+  constexpr bool TSA = WBF;  // expanded weights in tensor memory
+  using SM = GemmSmem<BN, CONV, SWAP, WBF ? wbf_katoms(BN) : 0, TSA>;
   static_assert(!W4 || SM::KA == 1, "int4 stages hold one K atom");
   constexpr int CW = SM::CW;
   pdl_launch_dependents();  // the grid is co-resident: dependents only take idle SMs
@@ -466,11 +465,7 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
               if (TSA) {
                 mma_bf16_ts(d, ta + j * (GEMM_BK / 4) + k * (GEMM_UMMA_K / 4), bd, IDESC, acc);
               } else {
-                const uint64_t ad = sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K);
-                if (WBF)
-                  mma_bf16(d, ad, bd, IDESC, acc);
-                else
-                  mma_s8(d, ad, bd, IDESC, acc);
+                mma_s8(d, sw128_kmajor_desc(sa + j * SM::A_ATOM + k * GEMM_UMMA_K), bd, IDESC, acc);
               }
             }
           }
@@ -881,10 +876,10 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
       }
     }
   } else if (CONV) {
-    // ------------------------------------------------------------ int4 unpack /
-    // int8 -> bf16 (WBF).  Each thread reads its share of every packed atom of
-    // the stage, the four warps meet (bounded), then each writes the expanded
-    // swizzled rows over the slot the packed bytes came in.
+    // ------------------------------------------------------------ int4 unpack
+    // Each thread reads its share of every packed atom of the stage, the four
+    // warps meet (bounded), then each writes the expanded swizzled rows over
+    // the slot the packed bytes came in.
     const int ct = threadIdx.x - 192;  // 0..127
     constexpr int WR = SM::W_ROWS;
     constexpr int PER = WR * 4 / 128;  // 16-byte packed pieces per thread and atom
@@ -934,14 +929,10 @@ __global__ void __launch_bounds__((W4 || WBF) ? 320 : 192) __maxnreg__((W4 || WB
           uint32_t o[8];
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            if (WBF) {
-              i8x4_to_bf16x4(w[h], o[2 * h], o[2 * h + 1]);
-            } else {
-              const uint32_t lo = (w[h] << 4) & 0xF0F0F0F0u;
-              const uint32_t hi = w[h] & 0xF0F0F0F0u;
-              o[2 * h] = __byte_perm(lo, hi, 0x5140);
-              o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
-            }
+            const uint32_t lo = (w[h] << 4) & 0xF0F0F0F0u;
+            const uint32_t hi = w[h] & 0xF0F0F0F0u;
+            o[2 * h] = __byte_perm(lo, hi, 0x5140);
+            o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
           }
           const int sw = r & 7;
           uint8_t* d0 = unp + r * 128 + (((2 * pc) ^ sw) << 4);
