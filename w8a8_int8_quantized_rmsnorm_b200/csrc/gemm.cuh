@@ -48,7 +48,7 @@ constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 128;  // int8 elements (bytes) of K per swizzle atom
 constexpr int GEMM_UMMA_K = 32;
 constexpr int GEMM_MAX_STAGES = 16;
-constexpr int GEMM_GROUP_A = 8;
+constexpr int GEMM_GROUP_A = 8;  // rasterisation group of the single-CTA kernels
 // decode kernels: before the dependency wait, the weights of this many K atoms
 // beyond the ring's first fill go towards L2
 constexpr int GEMM_PREFETCH_ATOMS = 8;
@@ -83,6 +83,7 @@ struct GemmArgs {
   int M, N, K;
   int rowsA, rowsB;  // rows of operands A and B
   int tilesA, tilesB;
+  int group_a;       // tiles run in groups of this many A tiles, all B tiles of a group first
   int num_tiles;
   int num_kb;        // pipeline stages of K per tile (KA atoms of 128 bytes each)
   int stages;
@@ -154,10 +155,10 @@ __device__ __forceinline__ int sk_begin_of(const GemmArgs& a, int c) {
 }
 
 __device__ __forceinline__ void tile_coords(const GemmArgs& a, int tile, int& ta, int& tb) {
-  const int per_group = GEMM_GROUP_A * a.tilesB;
+  const int per_group = a.group_a * a.tilesB;
   const int group = tile / per_group;
-  const int first = group * GEMM_GROUP_A;
-  const int ga = min(GEMM_GROUP_A, a.tilesA - first);
+  const int first = group * a.group_a;
+  const int ga = min(a.group_a, a.tilesA - first);
   const int local = tile - group * per_group;
   ta = first + local % ga;
   tb = local / ga;
