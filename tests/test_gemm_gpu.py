@@ -36,9 +36,11 @@ SHAPES = [
     # 256 x 256 tiles, a single wave of at most one tile per four-CTA cluster
     # splits K over two pairs, larger grids split by stream-K (520 x 3000: one
     # partial wave of 36 pair tiles; 2200 x 2248: a full wave of 74 and a tail
-    # of 7; both ragged in M, N and K)
+    # of 7; both ragged in M, N and K).  Decode shapes with more 128-row weight
+    # tiles than SMs (100 x 19000: ragged; 128 x 24576: the gate/up decode
+    # GEMM, all outputs)
     (1, 256, 512), (3, 136, 512), (16, 1024, 4096), (17, 264, 1040), (40, 512, 256),
-    (64, 128, 768), (100, 2056, 144), (128, 520, 4096),
+    (64, 128, 768), (100, 2056, 144), (128, 520, 4096), (100, 19000, 1040), (128, 24576, 4096),
     (129, 264, 512), (256, 512, 4096), (300, 1032, 1040), (512, 4096, 12288),
     (1024, 1024, 4096), (2048, 1536, 16), (777, 8, 32),
     (1280, 2560, 1088), (520, 3000, 1040), (2200, 2248, 4000), (2048, 4096, 1024),

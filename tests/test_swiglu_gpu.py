@@ -107,8 +107,10 @@ def test_fold_row_scales(cr):
 # ------------------------------------------------------------------ the GEMM
 SHAPES = [
     # (M, I, K): swapped operand roles for M <= 128, CTA pairs above; I = 48
-    # and 520 leave a partial 128- or 256-row weight tile
+    # and 520 leave a partial 128- or 256-row weight tile; (100, 9600): 19200
+    # weight rows, more 128-row decode tiles than SMs
     (1, 256, 512), (3, 48, 256), (16, 1024, 4096), (40, 528, 1040), (128, 2048, 4096),
+    (100, 9600, 1040),
     (129, 272, 512), (256, 1024, 4096), (300, 1040, 1040), (512, 1536, 4096),
 ]
 
