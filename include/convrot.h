@@ -280,13 +280,13 @@ convrot_status convrot_fold_row_scales(float* s_row, const float* smooth, int n,
  *   Xr[m,k] = bf16_rn(r * (x * (1 + norm_w)) * R)      convrot_rotate_act_bf16
  *             (norm_w NULL: no RMSNorm, r = 1; group 256, 16 or 0)
  *   Y[m,n]  = bf16_rn(s_row[n] * sum_k Xr[m,k] * Wq[n,k])   convrot_weight_only_linear
- * The int8 codes are expanded to bf16 (exactly) in shared memory and
+ * The int8 codes are expanded to bf16 (exactly) into tensor memory and
  * multiplied on the tensor cores (bf16 inputs, fp32 accumulation), so Y
  * approximates x W^T with the weight's int8 rounding only.
  * x bf16 [M, K], Xr bf16 [M, K], Wq int8 [N, K], s_row fp32 [N], Y bf16 [M, N];
  * K % 16 == 0, N % 8 == 0; all 16-byte aligned.
  * workspace: at least convrot_weight_only_workspace_bytes(M, N, K) bytes
- * (0: may be NULL), with the rules of convrot_int8_linear.  Decode shapes
+ * (0: may be NULL), with the rules of convrot_int8_linear.  Some shapes
  * split the K range of some output tiles over two CTAs; their fp32 partial
  * sums meet there, added at L2.  A tile never has more than two parts, and
  * 0 + a + b is the same in either order, so results do not depend on timing.
