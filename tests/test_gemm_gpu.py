@@ -44,6 +44,9 @@ SHAPES = [
     (129, 264, 512), (256, 512, 4096), (300, 1032, 1040), (512, 4096, 12288),
     (1024, 1024, 4096), (2048, 1536, 16), (777, 8, 32),
     (1280, 2560, 1088), (520, 3000, 1040), (2200, 2248, 4000),
+    # the decode GEMMs at full size (stream-K over 192 weight tiles, split tiles
+    # summed at L2), every output
+    (1, 24576, 4096), (16, 24576, 4096),
     # long K: the pair kernel rasterises in groups of as many 256-row activation
     # tiles as fit ~40 MB (here 5 of the 9, the second group partial)
     (2100, 1040, 32768),
@@ -110,7 +113,8 @@ def test_int8_linear_bf16(cr, M, N, K):
 
 
 PACK_SHAPES = [(1, 256, 512), (16, 1024, 4096), (33, 264, 1056), (128, 520, 4096),
-               (129, 264, 512), (512, 4096, 12288), (1000, 1032, 2080), (2100, 1040, 32768)]
+               (129, 264, 512), (512, 4096, 12288), (1000, 1032, 2080), (2100, 1040, 32768),
+               (4096, 4096, 4096)]
 
 
 def _rand_w4(N, K, seed):
